@@ -1,0 +1,159 @@
+// gl_api.cu -- the C ABI (include/gl.h): argument checks, then launches.
+// Nothing here allocates device memory or synchronises the host.
+#include "gl_internal.h"
+
+namespace {
+
+using gl::GemmCall;
+
+cudaStream_t to_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool grouped_ok(const gl_grouped& g, int G) {
+  if (g.mode == GL_STACKED) return g.base != nullptr;
+  if (g.mode == GL_PER_GROUP) {
+    if (g.ptrs == nullptr) return false;
+    for (int i = 0; i < G; ++i)
+      if (g.ptrs[i] == nullptr) return false;
+    return true;
+  }
+  return false;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool grouped_aligned(const gl_grouped& g, int G) {
+  if (g.mode == GL_STACKED) return aligned16(g.base);
+  for (int i = 0; i < G; ++i)
+    if (!aligned16(g.ptrs[i])) return false;
+  return true;
+}
+
+// Common shape checks for the three GEMMs (grouped_linear.py: in/out features
+// and group count must be positive; TMA needs 16-byte row pitches).
+gl_status check_gemm_dims(int G, int64_t M, int N, int K) {
+  if (G <= 0 || G > GL_MAX_GROUPS || M < 0 || N <= 0 || K <= 0) return GL_ERR_INVALID;
+  if ((N % 8) != 0 || (K % 8) != 0) return GL_ERR_UNSUPPORTED;
+  if (M >= (int64_t(1) << 31)) return GL_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  // persistent-scheduler tile counts are int32
+  const int64_t rt = (M + 127) / 128 + G;
+  const int64_t ct = (int64_t(N > K ? N : K) + 127) / 128;
+  if (rt * ct >= (int64_t(1) << 31) || int64_t(G) * ct * ct >= (int64_t(1) << 31)) return GL_ERR_UNSUPPORTED;
+  return GL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gl_version(void) { return 100; }
+
+const char* gl_status_string(gl_status s) {
+  switch (s) {
+    case GL_OK: return "ok";
+    case GL_ERR_INVALID: return "invalid argument";
+    case GL_ERR_UNSUPPORTED: return "unsupported size or alignment";
+    case GL_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+gl_status gl_offsets(const int64_t* m_splits, int G, int64_t expect_rows, int64_t out_rows,
+                     int64_t* offsets, int32_t* status, void* stream) {
+  if (m_splits == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if (G <= 0 || G > GL_MAX_GROUPS || expect_rows < 0 || out_rows < 0) return GL_ERR_INVALID;
+  return gl::launch_offsets(m_splits, G, expect_rows, out_rows, offsets, status, to_stream(stream));
+}
+
+gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int64_t* offsets,
+                 int32_t* status, int G, int64_t M, int N, int K, void* y, int64_t y_rows,
+                 void* stream) {
+  gl_status st = check_gemm_dims(G, M, N, K);
+  if (st != GL_OK) return st;
+  if (x == nullptr || y == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if (!grouped_ok(w, G) || (bias != nullptr && !grouped_ok(*bias, G))) return GL_ERR_INVALID;
+  if (y_rows < M) return GL_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(y) || !grouped_aligned(w, G) || (bias && !grouped_aligned(*bias, G)))
+    return GL_ERR_UNSUPPORTED;
+  GemmCall c{};
+  c.mode = gl::kFwd;
+  c.a = x;
+  c.w = w;
+  c.bias = bias;
+  c.out = y;
+  c.out_rows = y_rows;
+  c.offsets = offsets;
+  c.status = status;
+  c.G = G;
+  c.M = M;
+  c.N = N;
+  c.K = K;
+  c.stream = to_stream(stream);
+  return gl::launch_grouped_gemm(c);
+}
+
+gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t* status, int G,
+                   int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream) {
+  gl_status st = check_gemm_dims(G, M, N, K);
+  if (st != GL_OK) return st;
+  if (dy == nullptr || dx == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if (!grouped_ok(w, G)) return GL_ERR_INVALID;
+  if (dx_rows < M) return GL_ERR_INVALID;
+  if (!aligned16(dy) || !aligned16(dx) || !grouped_aligned(w, G)) return GL_ERR_UNSUPPORTED;
+  GemmCall c{};
+  c.mode = gl::kDgrad;
+  c.a = dy;
+  c.w = w;
+  c.out = dx;
+  c.out_rows = dx_rows;
+  c.offsets = offsets;
+  c.status = status;
+  c.G = G;
+  c.M = M;
+  c.N = N;
+  c.K = K;
+  c.stream = to_stream(stream);
+  return gl::launch_grouped_gemm(c);
+}
+
+gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_t* status, int G,
+                   int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream) {
+  gl_status st = check_gemm_dims(G, M, N, K);
+  if (st != GL_OK) return st;
+  if (x == nullptr || dy == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if (!grouped_ok(main_grad, G)) return GL_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(dy) || !grouped_aligned(main_grad, G)) return GL_ERR_UNSUPPORTED;
+  GemmCall c{};
+  c.mode = gl::kWgrad;
+  c.a = dy;
+  c.b = x;
+  c.out_grouped = main_grad;
+  c.offsets = offsets;
+  c.status = status;
+  c.G = G;
+  c.M = M;
+  c.N = N;
+  c.K = K;
+  c.accumulate = accumulate ? 1 : 0;
+  c.stream = to_stream(stream);
+  return gl::launch_grouped_gemm(c);
+}
+
+gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
+                               int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                               uint8_t* codes_c, uint8_t* scales_c, void* stream) {
+  if (src == nullptr || rows < 0 || cols <= 0 || G <= 0 || G > GL_MAX_GROUPS) return GL_ERR_INVALID;
+  if (codes_r == nullptr && codes_c == nullptr) return GL_ERR_INVALID;
+  if ((codes_r != nullptr) != (scales_r != nullptr) && codes_r != nullptr) return GL_ERR_INVALID;
+  if (codes_r != nullptr && scales_r == nullptr) return GL_ERR_INVALID;
+  if (codes_c != nullptr && scales_c == nullptr) return GL_ERR_INVALID;
+  if (cols % 32 != 0) return GL_ERR_UNSUPPORTED;
+  if (row_offsets == nullptr && rows % G != 0) return GL_ERR_INVALID;
+  if (!aligned16(src) || (codes_r && (reinterpret_cast<uintptr_t>(codes_r) & 7u)) ||
+      (codes_c && (reinterpret_cast<uintptr_t>(codes_c) & 7u)))
+    return GL_ERR_UNSUPPORTED;
+  if (rows == 0) return GL_OK;
+  return gl::launch_quantize(src, rows, cols, row_offsets, G, status, codes_r, scales_r, codes_c,
+                             scales_c, to_stream(stream));
+}
+
+}  // extern "C"

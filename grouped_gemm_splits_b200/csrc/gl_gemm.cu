@@ -1,0 +1,593 @@
+// gl_gemm.cu -- persistent ragged grouped GEMM on sm_100a tensor cores (bf16).
+//
+// One kernel template serves the three products of the grouped linear layer
+// (TransformerEngine ``grouped_linear.py``, ops/basic: fuser_forward "Perform
+// GEMMs" and fuser_backward "Perform dgrad GEMMs" / "Perform wgrad GEMMs"):
+//
+//   FWD    y[r, n]        = sum_k x[r, k]  W_g[n, k]   (+ b_g[n])   rows r of group g
+//   DGRAD  dx[r, k]       = sum_n dy[r, n] W_g[n, k]                rows r of group g
+//   WGRAD  main_grad_g[n,k] (+)= sum_{r in g} dy[r, n] x[r, k]
+//
+// Each CTA owns one SM.  Warp 0 streams operand tiles with TMA into a ring of
+// shared-memory stages, warp 1 issues tcgen05.mma (fp32 accumulators in
+// TMEM, two 128x256 accumulators so the epilogue of one tile overlaps the
+// main loop of the next) and warps 2-5 drain TMEM: bias + bf16 rounding and
+// row-clipped stores for FWD/DGRAD, TMA reduce-add (accumulate) or TMA store
+// (overwrite) of fp32 main_grad tiles for WGRAD.  Tiles are enumerated group
+// by group from the device offsets (a tile prefix built in shared memory), so
+// empty groups cost nothing and the host never learns the split sizes.
+#include <cuda_bf16.h>
+
+#include "gl_internal.h"
+#include "gl_ptx.cuh"
+
+namespace gl {
+namespace {
+
+constexpr int BM = 128;  // accumulator rows (TMEM lanes)
+constexpr int BN = 256;  // accumulator columns
+constexpr int BK = 64;   // contraction elements per stage (one 128-byte swizzle row)
+constexpr int kThreads = 192;
+constexpr int kPG = 64;  // per-group tensor maps carried by one launch
+
+template <int MODE>
+struct Cfg {
+  static constexpr int kStages = (MODE == kWgrad) ? 3 : 4;
+  static constexpr int kABytes = BM * BK * 2;  // 16 KB
+  static constexpr int kBBytes = BN * BK * 2;  // 32 KB
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStagingBytes = (MODE == kWgrad) ? 2 * BM * 32 * 4 : 0;  // 2 x 16 KB
+  static constexpr int kBarOffset = kStages * kStageBytes + kStagingBytes;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kPrefixOffset = kBarOffset + kBarBytes;
+  // A / B operand storage in shared memory: 1 = MN-major (see file header)
+  static constexpr int kAMN = (MODE == kWgrad) ? 1 : 0;
+  static constexpr int kBMN = (MODE == kFwd) ? 0 : 1;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, kAMN, kBMN);
+};
+
+struct GemmParams {
+  CUtensorMap tmA;    // FWD x{K,M} box{64,128}; DGRAD dy{N,M} box{64,128}; WGRAD dy{N,M} box{64,64}
+  CUtensorMap tmB;    // stacked W{K,N,G}: FWD box{64,256,1}, DGRAD box{64,64,1}; WGRAD x{K,M} box{64,64}
+  CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,128,1}
+  const int64_t* offsets;  // G+1 entries
+  int32_t* status;
+  int64_t M;
+  int64_t out_rows;
+  void* out;                  // FWD y / DGRAD dx (bf16)
+  const __nv_bfloat16* bias;  // stacked bias [G,N] or null
+  int G;
+  int N, K;
+  int has_bias;
+  int accumulate;
+};
+
+template <bool PG>
+struct PGArgs {
+  CUtensorMap tm[kPG];  // FWD/DGRAD: W_g{K,N}; WGRAD: main_grad_g{K,N}
+  const __nv_bfloat16* bias[kPG];
+  __device__ const CUtensorMap* map(int g) const { return &tm[g]; }
+  __device__ const __nv_bfloat16* b(int g) const { return bias[g]; }
+};
+template <>
+struct PGArgs<false> {
+  int unused;
+  __device__ const CUtensorMap* map(int) const { return nullptr; }
+  __device__ const __nv_bfloat16* b(int) const { return nullptr; }
+};
+
+struct Tile {
+  int g;
+  int num_kb;
+  int mt, nt;
+  int64_t r0, r1;  // FWD/DGRAD: output rows [r0, r1) clip; WGRAD: contraction rows [r0, r1)
+};
+
+__device__ __forceinline__ int ceil_div_i(int64_t a, int b) { return static_cast<int>((a + b - 1) / b); }
+
+template <int MODE>
+__device__ __forceinline__ int tiles_of_group(int64_t m, const GemmParams& p) {
+  if (MODE == kFwd) return m > 0 ? ceil_div_i(m, BM) * ceil_div_i(p.N, BN) : 0;
+  if (MODE == kDgrad) return m > 0 ? ceil_div_i(m, BM) * ceil_div_i(p.K, BN) : 0;
+  return (m > 0 || !p.accumulate) ? ceil_div_i(p.N, BM) * ceil_div_i(p.K, BN) : 0;
+}
+
+template <int MODE>
+__device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const GemmParams& p) {
+  // largest g with prefix[g] <= t (prefix is non-decreasing, prefix[0] = 0)
+  int lo = 0, hi = p.G;  // answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= t) lo = mid; else hi = mid;
+  }
+  Tile tl;
+  tl.g = lo;
+  const int local = t - prefix[lo];
+  const int64_t o0 = __ldg(p.offsets + lo), o1 = __ldg(p.offsets + lo + 1);
+  const int64_t m = o1 > o0 ? o1 - o0 : 0;
+  if (MODE == kWgrad) {
+    const int mtn = ceil_div_i(p.N, BM);
+    tl.mt = local % mtn;
+    tl.nt = local / mtn;
+    tl.r0 = o0;
+    tl.r1 = o0 + m;
+    tl.num_kb = ceil_div_i(m, BK);
+  } else {
+    const int mtg = ceil_div_i(m, BM);
+    tl.mt = local % mtg;  // m-tiles fastest: neighbouring CTAs share a weight strip
+    tl.nt = local / mtg;
+    tl.r0 = o0 + static_cast<int64_t>(tl.mt) * BM;
+    tl.r1 = o0 + m;
+    tl.num_kb = ceil_div_i(MODE == kFwd ? p.K : p.N, BK);
+  }
+  return tl;
+}
+
+__device__ __forceinline__ void report_abort(volatile int* abort_flag, int32_t* status) {
+  if (!*abort_flag) {
+    *abort_flag = 1;
+    if (status) atomicOr(status, GL_DEV_TIMEOUT);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), round to nearest even
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int MODE, bool PG>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ PGArgs<PG> pg) {
+  using C = Cfg<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* skip_flag = abort_flag + 1;
+  int* prefix = reinterpret_cast<int*>(smem + C::kPrefixOffset);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *skip_flag = (p.status != nullptr && *reinterpret_cast<volatile int32_t*>(p.status) != 0) ? 1 : 0;
+    *abort_flag = 0;
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(mma_done, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (*skip_flag) return;  // bad split sizes reported by gl_offsets: write nothing
+
+  if (warp == 0) {
+    // tile prefix over groups: prefix[g] = number of tiles of groups < g
+    int carry = 0;
+    for (int base = 0; base < p.G; base += 32) {
+      const int i = base + lane;
+      int cnt = 0;
+      if (i < p.G) {
+        const int64_t m = __ldg(p.offsets + i + 1) - __ldg(p.offsets + i);
+        cnt = tiles_of_group<MODE>(m, p);
+      }
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, cnt, off);
+        if (lane >= off) cnt += v;
+      }
+      if (i < p.G) prefix[i + 1] = carry + cnt;
+      carry += __shfl_sync(0xffffffffu, cnt, 31);
+    }
+    if (lane == 0) prefix[0] = 0;
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * BN);  // two 128 x 256 fp32 accumulators = all 512 columns
+    tmem_relinquish();
+  } else if (warp == 2 && lane == 0) {
+    tma_prefetch_desc(&p.tmA);
+    if (!PG) tma_prefetch_desc(&p.tmB);
+    if (MODE == kWgrad) tma_prefetch_desc(PG ? pg.map(0) : &p.tmOut);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = prefix[p.G];
+
+  if (warp == 0) {
+    // ===================== TMA producer =====================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+        const Tile tl = decode_tile<MODE>(t, prefix, p);
+        for (int kb = 0; kb < tl.num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { report_abort(abort_flag, p.status); break; }
+          uint8_t* sa = smem + stage * C::kStageBytes;
+          uint8_t* sb = sa + C::kABytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          if (MODE == kFwd) {
+            tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0));
+            if (PG) tma_load_2d(sb, pg.map(tl.g), &full[stage], kb * BK, tl.nt * BN);
+            else    tma_load_3d(sb, &p.tmB, &full[stage], kb * BK, tl.nt * BN, tl.g);
+          } else if (MODE == kDgrad) {
+            tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0));
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c) {
+              if (PG) tma_load_2d(sb + c * 8192, pg.map(tl.g), &full[stage], tl.nt * BN + c * 64, kb * BK);
+              else    tma_load_3d(sb + c * 8192, &p.tmB, &full[stage], tl.nt * BN + c * 64, kb * BK, tl.g);
+            }
+          } else {
+            const int32_t row = static_cast<int32_t>(tl.r0 + kb * BK);
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(sa + c * 8192, &p.tmA, &full[stage], tl.mt * BM + c * 64, row);
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(sb + c * 8192, &p.tmB, &full[stage], tl.nt * BN + c * 64, row);
+          }
+          ++issued;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Do not leave while a TMA load may still be writing shared memory.
+      const int inflight = issued < C::kStages ? issued : C::kStages;
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < inflight; ++i) {
+        if (--s < 0) { s = C::kStages - 1; ph ^= 1u; }
+        mbar_wait_bounded(&full[s], ph);
+      }
+    }
+  } else if (warp == 1) {
+    // ===================== MMA issuer =====================
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const Tile tl = decode_tile<MODE>(t, prefix, p);
+      const int buf = it & 1;
+      const uint32_t tph = (it >> 1) & 1;
+      // every lane waits; the warp acts on a unanimous result
+      if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], tph ^ 1u, abort_flag))) {
+        report_abort(abort_flag, p.status);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + buf * BN;
+      bool ok = true;
+      for (int kb = 0; kb < tl.num_kb; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+          report_abort(abort_flag, p.status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* sa = smem + stage * C::kStageBytes;
+        uint8_t* sb = sa + C::kABytes;
+        int ksteps = BK / 16;
+        if (MODE == kWgrad && kb == tl.num_kb - 1) {
+          // Ragged contraction: rows past the group's end must not contribute.
+          // Skip whole 16-row MMA steps beyond the end and zero the rows of the
+          // last partial step in both operands.
+          const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
+          if (valid < BK) {
+            ksteps = (valid + 15) >> 4;
+            const int zend = ksteps * 16;
+            const int nrows = zend - valid;
+            if (nrows > 0) {
+              // 6 chunks (2 of A, 4 of B) of [64 rows x 128 B]; 8 x 16 B per row
+              const int per_chunk = nrows * 8;
+              for (int idx = lane; idx < 6 * per_chunk; idx += 32) {
+                const int chunk = idx / per_chunk;
+                const int rem = idx - chunk * per_chunk;
+                const int row = valid + (rem >> 3);
+                uint8_t* base = (chunk < 2) ? (sa + chunk * 8192) : (sb + (chunk - 2) * 8192);
+                *reinterpret_cast<uint4*>(base + row * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
+          for (int ks = 0; ks < ksteps; ++ks) {
+            uint64_t ad, bd;
+            if (C::kAMN) ad = smem_desc_sw128(a0 + ks * 2048, 8192, 1024);
+            else         ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
+            if (C::kBMN) bd = smem_desc_sw128(b0 + ks * 2048, 8192, 1024);
+            else         bd = smem_desc_sw128(b0 + ks * 32, 16, 1024);
+            mma_bf16_ss(d_tmem, ad, bd, C::kIdesc, (kb > 0 || ks > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+        }
+        __syncwarp();
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        if (tl.num_kb > 0) tc_commit(&tfull[buf]);
+        else mbar_arrive(&tfull[buf]);  // nothing accumulated: epilogue writes zeros
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      tc_commit(mma_done);  // all MMAs issued by this thread have completed
+      mbar_wait_bounded(mma_done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ===================== epilogue (warps 2..5) =====================
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    const bool issuer = (warp == 2 && lane == 0);
+    int it = 0;
+    int chunk_ctr = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const Tile tl = decode_tile<MODE>(t, prefix, p);
+      const int buf = it & 1;
+      const uint32_t tph = (it >> 1) & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
+      if (!ok) report_abort(abort_flag, p.status);
+      if (MODE == kWgrad) {
+        // all four warps must agree before any named barrier below
+        uint32_t bad;
+        asm volatile(
+            "{\n\t.reg .pred P, Q;\n\t"
+            "setp.ne.b32 P, %1, 0;\n\t"
+            "bar.red.or.pred Q, 1, 128, P;\n\t"
+            "selp.b32 %0, 1, 0, Q;\n\t}"
+            : "=r"(bad)
+            : "r"((!ok || *abort_flag) ? 1 : 0));
+        if (bad) break;
+      } else if (!ok) {
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + buf * BN + (static_cast<uint32_t>(q * 32) << 16);
+
+      if (MODE != kWgrad) {
+        const int Nout = (MODE == kFwd) ? p.N : p.K;
+        const int64_t row = tl.r0 + row_in_tile;
+        const bool row_ok = row >= 0 && row < tl.r1 && row < p.out_rows;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+        const __nv_bfloat16* bias = nullptr;
+        if (MODE == kFwd && p.has_bias)
+          bias = PG ? pg.b(tl.g) : (p.bias + static_cast<int64_t>(tl.g) * p.N);
+        const int nchunks = min(BN / 32, ceil_div_i(Nout - tl.nt * BN, 32));
+        for (int c = 0; c < nchunks; ++c) {
+          const int n = tl.nt * BN + c * 32;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tacc + c * 32, r);
+          tmem_ld_wait();
+          if (c == nchunks - 1) {
+            // accumulator fully read: hand the buffer back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);
+          }
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if (bias != nullptr) {
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+              if (n + j8 * 8 < Nout) {
+                const uint4 bv = __ldg(reinterpret_cast<const uint4*>(bias + n + j8 * 8));
+                const __nv_bfloat16* bb = reinterpret_cast<const __nv_bfloat16*>(&bv);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j8 * 8 + j] += __bfloat162float(bb[j]);
+              }
+            }
+          }
+          if (row_ok) {
+            __nv_bfloat16* dst = out + row * static_cast<int64_t>(Nout) + n;
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+              if (n + j8 * 8 < Nout) {
+                uint4 w;
+                w.x = pack_bf16x2(v[j8 * 8 + 0], v[j8 * 8 + 1]);
+                w.y = pack_bf16x2(v[j8 * 8 + 2], v[j8 * 8 + 3]);
+                w.z = pack_bf16x2(v[j8 * 8 + 4], v[j8 * 8 + 5]);
+                w.w = pack_bf16x2(v[j8 * 8 + 6], v[j8 * 8 + 7]);
+                *reinterpret_cast<uint4*>(dst + j8 * 8) = w;
+              }
+            }
+          }
+        }
+        if (nchunks <= 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+      } else {
+        // main_grad tile: rows n0.. (TMEM lanes) x cols k0.. (TMEM columns)
+        float* staging = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
+        const int n0 = tl.mt * BM;
+        const int k0 = tl.nt * BN;
+        const int nchunks = min(BN / 32, ceil_div_i(p.K - k0, 32));
+        const bool have_acc = tl.num_kb > 0;
+        for (int c = 0; c < nchunks; ++c, ++chunk_ctr) {
+          float* stg = staging + (chunk_ctr & 1) * (BM * 32);
+          if (issuer) bulk_wait_group_read<1>();  // the buffer's previous store has read it
+          named_barrier_sync(1, 128);
+          uint32_t r[32];
+          if (have_acc) {
+            tmem_ld_32x32b_x32(tacc + c * 32, r);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = 0u;
+          }
+          if (c == nchunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);
+          }
+          // row `row_in_tile` of a [128 x 32] fp32 box, 128-byte swizzle
+          uint8_t* rowp = reinterpret_cast<uint8_t*>(stg) + row_in_tile * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int pj = j ^ (row_in_tile & 7);
+            *reinterpret_cast<uint4*>(rowp + pj * 16) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+          }
+          fence_proxy_async_smem();
+          named_barrier_sync(1, 128);
+          if (issuer) {
+            const int kc = k0 + c * 32;
+            if (PG) {
+              if (p.accumulate) tma_reduce_add_2d(pg.map(tl.g), stg, kc, n0);
+              else              tma_store_2d(pg.map(tl.g), stg, kc, n0);
+            } else {
+              if (p.accumulate) tma_reduce_add_3d(&p.tmOut, stg, kc, n0, tl.g);
+              else              tma_store_3d(&p.tmOut, stg, kc, n0, tl.g);
+            }
+            bulk_commit_group();
+          }
+        }
+        if (nchunks <= 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+      }
+    }
+    if (MODE == kWgrad && issuer) bulk_wait_group<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * BN);
+  }
+}
+
+template <int MODE>
+constexpr int smem_bytes_for(int G) {
+  return Cfg<MODE>::kPrefixOffset + (G + 1) * 4 + 1024;  // + alignment slack
+}
+
+bool make_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_in,
+             uint32_t box_out, CUtensorMapDataType dt, int esize) {
+  const uint64_t dims[2] = {inner, outer};
+  const uint64_t strides[1] = {inner * esize};
+  const uint32_t box[2] = {box_in, box_out};
+  return encode_tmap(m, dt, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool make_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+             uint32_t box_in, uint32_t box_mid, CUtensorMapDataType dt, int esize) {
+  const uint64_t dims[3] = {inner, mid, outer};
+  const uint64_t strides[2] = {inner * esize, inner * mid * esize};
+  const uint32_t box[3] = {box_in, box_mid, 1};
+  return encode_tmap(m, dt, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int MODE, bool PG>
+gl_status launch_one(const GemmParams& prm, const PGArgs<PG>& pga, int G, cudaStream_t stream) {
+  const int smem = smem_bytes_for<MODE>(G);
+  auto kern = grouped_gemm_kernel<MODE, PG>;
+  if (set_max_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return GL_ERR_CUDA;
+  kern<<<num_sms(), kThreads, smem, stream>>>(prm, pga);
+  return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
+}
+
+template <int MODE>
+gl_status launch_mode(const GemmCall& c) {
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  GemmParams prm;
+  memset(&prm, 0, sizeof(prm));
+  prm.status = c.status;
+  prm.M = c.M;
+  prm.out_rows = c.out_rows;
+  prm.out = c.out;
+  prm.N = c.N;
+  prm.K = c.K;
+  prm.accumulate = c.accumulate;
+  prm.has_bias = (MODE == kFwd && c.bias != nullptr) ? 1 : 0;
+  const uint64_t Mrows = c.M > 0 ? static_cast<uint64_t>(c.M) : 1;  // a map needs >= 1 row
+  bool ok = true;
+  if (MODE == kFwd) {
+    ok &= make_2d(&prm.tmA, c.a, c.K, Mrows, BK, BM, BF, 2);
+  } else if (MODE == kDgrad) {
+    ok &= make_2d(&prm.tmA, c.a, c.N, Mrows, BK, BM, BF, 2);
+  } else {
+    ok &= make_2d(&prm.tmA, c.a, c.N, Mrows, 64, BK, BF, 2);
+    ok &= make_2d(&prm.tmB, c.b, c.K, Mrows, 64, BK, BF, 2);
+  }
+  if (!ok) return GL_ERR_UNSUPPORTED;
+
+  const bool stacked = (MODE == kWgrad) ? (c.out_grouped.mode == GL_STACKED) : (c.w.mode == GL_STACKED);
+  const bool bias_stacked = prm.has_bias && c.bias->mode == GL_STACKED;
+  if (stacked && (!prm.has_bias || bias_stacked)) {
+    if (MODE == kFwd) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, BK, BN, BF, 2);
+    if (MODE == kDgrad) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, 64, BK, BF, 2);
+    if (MODE == kWgrad)
+      ok &= make_3d(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 32, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+    if (!ok) return GL_ERR_UNSUPPORTED;
+    prm.offsets = c.offsets;
+    prm.G = c.G;
+    if (prm.has_bias) prm.bias = reinterpret_cast<const __nv_bfloat16*>(c.bias->base);
+    PGArgs<false> none{0};
+    return launch_one<MODE, false>(prm, none, c.G, c.stream);
+  }
+  // Per-group pointers (weights, biases or main_grad): launches of <= kPG groups.
+  PGArgs<true>* pga = new PGArgs<true>;
+  gl_status st = GL_OK;
+  for (int g0 = 0; g0 < c.G && st == GL_OK; g0 += kPG) {
+    const int cg = (c.G - g0) < kPG ? (c.G - g0) : kPG;
+    memset(pga, 0, sizeof(*pga));
+    for (int i = 0; i < cg; ++i) {
+      const int g = g0 + i;
+      if (MODE == kFwd || MODE == kDgrad) {
+        const void* wp = (c.w.mode == GL_STACKED)
+                             ? static_cast<const uint8_t*>(c.w.base) + static_cast<size_t>(g) * c.N * c.K * 2
+                             : c.w.ptrs[g];
+        if (MODE == kFwd) ok &= make_2d(&pga->tm[i], wp, c.K, c.N, BK, BN, BF, 2);
+        else              ok &= make_2d(&pga->tm[i], wp, c.K, c.N, 64, BK, BF, 2);
+        if (prm.has_bias)
+          pga->bias[i] = reinterpret_cast<const __nv_bfloat16*>(
+              c.bias->mode == GL_STACKED
+                  ? static_cast<const uint8_t*>(c.bias->base) + static_cast<size_t>(g) * c.N * 2
+                  : c.bias->ptrs[g]);
+      } else {
+        const void* gp = (c.out_grouped.mode == GL_STACKED)
+                             ? static_cast<const uint8_t*>(c.out_grouped.base) + static_cast<size_t>(g) * c.N * c.K * 4
+                             : c.out_grouped.ptrs[g];
+        ok &= make_2d(&pga->tm[i], gp, c.K, c.N, 32, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+      }
+    }
+    if (!ok) { st = GL_ERR_UNSUPPORTED; break; }
+    prm.offsets = c.offsets + g0;
+    prm.G = cg;
+    st = launch_one<MODE, true>(prm, *pga, cg, c.stream);
+  }
+  delete pga;
+  return st;
+}
+
+}  // namespace
+
+gl_status launch_grouped_gemm(const GemmCall& c) {
+  switch (c.mode) {
+    case kFwd: return launch_mode<kFwd>(c);
+    case kDgrad: return launch_mode<kDgrad>(c);
+    case kWgrad: return launch_mode<kWgrad>(c);
+  }
+  return GL_ERR_INVALID;
+}
+
+}  // namespace gl

@@ -1,0 +1,54 @@
+// gl_internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/gl.h"
+
+namespace gl {
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.  Returns
+// false if the driver rejected the map.  dims/strides are innermost first;
+// strides_bytes has rank-1 entries (dims 1..rank-1).
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                 CUtensorMapSwizzle swizzle);
+
+// Opt a kernel into more than 48 KB of dynamic shared memory (once).
+cudaError_t set_max_smem(const void* func, int bytes);
+
+enum GemmMode { kFwd = 0, kDgrad = 1, kWgrad = 2 };
+
+struct GemmCall {
+  int mode;
+  const void* a;           // FWD: x   DGRAD: dy   WGRAD: dy
+  const void* b;           // WGRAD: x (unused otherwise)
+  gl_grouped w;            // FWD/DGRAD weights
+  const gl_grouped* bias;  // FWD bias (nullable)
+  gl_grouped out_grouped;  // WGRAD main_grad
+  void* out;               // FWD y / DGRAD dx
+  int64_t out_rows;
+  const int64_t* offsets;
+  int32_t* status;
+  int G;
+  int64_t M;
+  int N, K;
+  int accumulate;
+  cudaStream_t stream;
+};
+
+gl_status launch_grouped_gemm(const GemmCall& c);
+
+gl_status launch_offsets(const int64_t* m, int G, int64_t expect_rows, int64_t out_rows,
+                         int64_t* offsets, int32_t* status, cudaStream_t stream);
+
+gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
+                          int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                          uint8_t* codes_c, uint8_t* scales_c, cudaStream_t stream);
+
+}  // namespace gl

@@ -1,0 +1,202 @@
+"""Python binding of ``libgl.so`` (see ``include/gl.h``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of the library.  PyTorch supplies device memory and the current
+stream.  The entry points keep the C names: :func:`gl_offsets`,
+:func:`gl_fwd`, :func:`gl_dgrad`, :func:`gl_wgrad` and
+:func:`group_quantize_mxfp8`.  There is no fallback: if the library has not
+been built, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Union
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgl.so")
+_lib = None
+
+GL_OK, GL_ERR_INVALID, GL_ERR_UNSUPPORTED, GL_ERR_CUDA = 0, 1, 2, 3
+GL_DEV_NEG_SPLIT, GL_DEV_SUM_MISMATCH, GL_DEV_OUT_OVERFLOW, GL_DEV_TIMEOUT = 1, 2, 4, 8
+GL_STACKED, GL_PER_GROUP = 0, 1
+
+EXPORTED = ("gl_version", "gl_status_string", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
+            "group_quantize_mxfp8")
+
+
+class GlGrouped(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("base", ctypes.c_void_p),
+                ("ptrs", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class GlError(RuntimeError):
+    pass
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load libgl.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise GlError(f"{_LIB_PATH} is missing: build it with `python -m grouped_gemm_splits_b200.build`")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    L.gl_version.restype = i32
+    L.gl_status_string.restype = ctypes.c_char_p
+    L.gl_status_string.argtypes = [i32]
+    L.gl_offsets.restype = i32
+    L.gl_offsets.argtypes = [vp, i32, i64, i64, vp, vp, vp]
+    L.gl_fwd.restype = i32
+    L.gl_fwd.argtypes = [vp, GlGrouped, ctypes.POINTER(GlGrouped), vp, vp, i32, i64, i32, i32, vp, i64, vp]
+    L.gl_dgrad.restype = i32
+    L.gl_dgrad.argtypes = [vp, GlGrouped, vp, vp, i32, i64, i32, i32, vp, i64, vp]
+    L.gl_wgrad.restype = i32
+    L.gl_wgrad.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, vp]
+    L.group_quantize_mxfp8.restype = i32
+    L.group_quantize_mxfp8.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, vp, vp, vp]
+    _lib = L
+    return L
+
+
+def _check(st: int, what: str) -> None:
+    if st != GL_OK:
+        raise GlError(f"{what}: {load().gl_status_string(st).decode()} ({st})")
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+TensorOrList = Union[torch.Tensor, Sequence[torch.Tensor]]
+
+
+def _grouped(t: TensorOrList, G: int):
+    """gl_grouped for a stacked tensor or a list of per-group tensors.
+
+    Returns (struct, keepalive) -- keep the second value alive for the call.
+    """
+    if isinstance(t, torch.Tensor):
+        assert t.is_contiguous() and t.shape[0] == G
+        return GlGrouped(GL_STACKED, t.data_ptr(), None), None
+    assert len(t) == G
+    arr = (ctypes.c_void_p * G)(*[x.data_ptr() for x in t])
+    return GlGrouped(GL_PER_GROUP, None, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))), arr
+
+
+def _shape_nk(w: TensorOrList):
+    return tuple((w if isinstance(w, torch.Tensor) else w[0]).shape[-2:])
+
+
+def gl_offsets(m_splits: torch.Tensor, expect_rows: int, out_rows: Optional[int] = None,
+               offsets: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
+    """Device prefix scan of ``m_splits`` (int64[G]) -> (offsets int64[G+1], status int32[1])."""
+    G = m_splits.numel()
+    dev = m_splits.device
+    if offsets is None:
+        offsets = torch.empty(G + 1, dtype=torch.int64, device=dev)
+    if status is None:
+        status = torch.empty(1, dtype=torch.int32, device=dev)
+    out_rows = expect_rows if out_rows is None else out_rows
+    _check(load().gl_offsets(m_splits.data_ptr(), G, expect_rows, out_rows, offsets.data_ptr(),
+                             status.data_ptr(), _stream()), "gl_offsets")
+    return offsets, status
+
+
+def gl_fwd(x: torch.Tensor, w: TensorOrList, bias: Optional[TensorOrList], offsets: torch.Tensor,
+           status: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y rows of group g = x rows of group g @ W_g^T (+ b_g).  ``y`` may be a
+    caller buffer with more rows than x; only the valid rows are written."""
+    G = offsets.numel() - 1
+    M, K = x.shape
+    N, K2 = _shape_nk(w)
+    assert K2 == K
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    wg, keep_w = _grouped(w, G)
+    bptr = None
+    keep_b = None
+    if bias is not None:
+        bg, keep_b = _grouped(bias, G)
+        bptr = ctypes.pointer(bg)
+    _check(load().gl_fwd(x.data_ptr(), wg, bptr, offsets.data_ptr(), status.data_ptr(), G, M, N, K,
+                         y.data_ptr(), y.shape[0], _stream()), "gl_fwd")
+    del keep_w, keep_b
+    return y
+
+
+def gl_dgrad(dy: torch.Tensor, w: TensorOrList, offsets: torch.Tensor, status: torch.Tensor,
+             dx: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """dx rows of group g = dy rows of group g @ W_g."""
+    G = offsets.numel() - 1
+    M, N = dy.shape
+    N2, K = _shape_nk(w)
+    assert N2 == N
+    if dx is None:
+        dx = torch.empty(M, K, dtype=torch.bfloat16, device=dy.device)
+    wg, keep_w = _grouped(w, G)
+    _check(load().gl_dgrad(dy.data_ptr(), wg, offsets.data_ptr(), status.data_ptr(), G, M, N, K,
+                           dx.data_ptr(), dx.shape[0], _stream()), "gl_dgrad")
+    del keep_w
+    return dx
+
+
+def gl_wgrad(x: torch.Tensor, dy: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
+             main_grad: TensorOrList, accumulate: bool = True) -> TensorOrList:
+    """main_grad[g] (+)= dy_g^T @ x_g (fp32)."""
+    G = offsets.numel() - 1
+    M, K = x.shape
+    N = dy.shape[1]
+    mg, keep = _grouped(main_grad, G)
+    _check(load().gl_wgrad(x.data_ptr(), dy.data_ptr(), offsets.data_ptr(), status.data_ptr(), G,
+                           M, N, K, mg, 1 if accumulate else 0, _stream()), "gl_wgrad")
+    del keep
+    return main_grad
+
+
+def colwise_scale_rows_bound(rows: int, G: int) -> int:
+    """Rows to allocate for columnwise scales: ceil(rows/32) + G."""
+    return (rows + 31) // 32 + G
+
+
+def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] = None, G: int = 1,
+                         rowwise: bool = True, colwise: bool = False,
+                         status: Optional[torch.Tensor] = None, out: Optional[dict] = None) -> dict:
+    """MXFP8 cast of a bf16 [rows, cols] tensor (rows in G groups).
+
+    Returns a dict with ``codes_r``/``scales_r`` (blocks along each row) and/or
+    ``codes_c``/``scales_c`` (blocks of 32 rows inside each group).
+    """
+    if src.dim() == 3:
+        G = src.shape[0]
+        src2 = src.reshape(-1, src.shape[-1])
+    else:
+        src2 = src
+    rows, cols = src2.shape
+    if row_offsets is not None:
+        G = row_offsets.numel() - 1
+    dev = src.device
+    out = {} if out is None else out
+    if rowwise:
+        out.setdefault("codes_r", torch.empty(rows, cols, dtype=torch.uint8, device=dev))
+        out.setdefault("scales_r", torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev))
+    if colwise:
+        out.setdefault("codes_c", torch.empty(rows, cols, dtype=torch.uint8, device=dev))
+        out.setdefault("scales_c", torch.empty(colwise_scale_rows_bound(rows, G), cols,
+                                               dtype=torch.uint8, device=dev))
+    _check(load().group_quantize_mxfp8(
+        src2.data_ptr(), rows, cols, _ptr(row_offsets), G, _ptr(status),
+        _ptr(out.get("codes_r")) if rowwise else None, _ptr(out.get("scales_r")) if rowwise else None,
+        _ptr(out.get("codes_c")) if colwise else None, _ptr(out.get("scales_c")) if colwise else None,
+        _stream()), "group_quantize_mxfp8")
+    return out

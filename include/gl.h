@@ -1,0 +1,193 @@
+/*
+ * gl.h -- C ABI of the B200 grouped linear library (libgl.so).
+ *
+ * The operation is the grouped (mixture-of-experts) linear layer of
+ * TransformerEngine's ``grouped_linear.py`` (ops/basic), ``GroupedLinear``:
+ * the input rows are split by ``m_splits`` into G contiguous groups and group
+ * i is multiplied by its own weight W_i, y_i = x_i W_i^T + b_i.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensors are row-major and contiguous; pointers named "device" point
+ *    to memory of the current CUDA device; the caller owns every buffer.  The
+ *    library never allocates device or pinned memory.
+ *  - Shapes: x [M,K], W_i [N,K], b_i [N], y [y_rows,N], dy [M,N],
+ *    dx [dx_rows,K], main_grad_i [N,K] fp32.  Group i owns rows
+ *    [o[i], o[i+1]) of x, y, dy and dx, where o = offsets from gl_offsets.
+ *  - Floating types: x, W, b, dy, y, dx are bf16 (2 bytes); main_grad is
+ *    fp32.  Products accumulate in fp32 on the tensor cores.
+ *  - Every call is asynchronous on ``stream`` (a cudaStream_t; NULL is the
+ *    legacy default stream) and never synchronises the host: split sizes stay
+ *    on the device.
+ *  - Host-checkable errors (null pointers, non-positive or unaligned sizes,
+ *    buffers too small) return GL_ERR_INVALID / GL_ERR_UNSUPPORTED before
+ *    anything is launched.  Data-dependent errors (negative split sizes, a
+ *    split sum that does not match M, more rows than the output buffer holds)
+ *    are detected on the device by gl_offsets, which writes them into the
+ *    int32 device status word; every later kernel that is given the status
+ *    word reads it first and writes nothing when it is non-zero.  A kernel
+ *    that gives up on a bounded internal wait ORs GL_DEV_TIMEOUT into it.
+ *    The caller reads the status word whenever it likes (for example with a
+ *    device-to-host copy after the step).
+ *  - Weights, biases and main_grad are passed as a gl_grouped: either one
+ *    stacked [G, rows, cols] tensor (the single grouped parameter of
+ *    ``GroupedLinear(single_grouped_weight=True)``) or a host array of G
+ *    device pointers, one [rows, cols] tensor per group (``weight0`` ..
+ *    ``weight{G-1}``).
+ */
+#ifndef GL_H_
+#define GL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- host return codes -------------------------------------------------- */
+typedef int gl_status;
+#define GL_OK 0
+#define GL_ERR_INVALID 1      /* bad argument; nothing was launched            */
+#define GL_ERR_UNSUPPORTED 2  /* valid but outside the kernels' limits (sizes  */
+                              /* not multiples of 8 / 32, too many groups ...) */
+#define GL_ERR_CUDA 3         /* a CUDA runtime call or a launch failed        */
+
+/* ---- device status word bits (int32, written by gl_offsets) ------------- */
+#define GL_DEV_NEG_SPLIT 1    /* some m_splits[i] < 0                          */
+#define GL_DEV_SUM_MISMATCH 2 /* sum(m_splits) != expect_rows                  */
+#define GL_DEV_OUT_OVERFLOW 4 /* sum(m_splits) > out_rows                      */
+#define GL_DEV_TIMEOUT 8      /* a kernel abandoned a bounded wait             */
+
+/* ---- grouped parameter descriptor --------------------------------------- */
+#define GL_STACKED 0   /* base -> [G, rows, cols], group stride rows*cols      */
+#define GL_PER_GROUP 1 /* ptrs -> host array of G device pointers [rows,cols] */
+
+typedef struct gl_grouped {
+  int mode;                /* GL_STACKED or GL_PER_GROUP                      */
+  const void* base;        /* GL_STACKED: device pointer                      */
+  const void* const* ptrs; /* GL_PER_GROUP: host array of G device pointers   */
+} gl_grouped;
+
+/* Largest G accepted by any entry point. */
+#define GL_MAX_GROUPS 4096
+
+/* Library version (major*10000 + minor*100 + patch). */
+int gl_version(void);
+
+/* Human-readable text of a gl_status value. */
+const char* gl_status_string(gl_status s);
+
+/*
+ * gl_offsets -- group row offsets from the split sizes, on the device.
+ *
+ * Computes o[0] = 0 and o[i+1] = o[i] + m_splits[i] (int64, G+1 values),
+ * the prefix sum with a leading zero that TransformerEngine's nvte_cumsum
+ * produces ("Single parameter for GroupedLinear module", PR #2727), so that the
+ * split sizes never travel to the host (``grouped_linear.py`` fuser_forward
+ * reads them with ``split_sizes.tolist()``, a host synchronisation).
+ *
+ *   m_splits    device int64[G], group row counts
+ *   G           1 <= G <= GL_MAX_GROUPS
+ *   expect_rows rows of the input (M); sum(m) must equal it
+ *   out_rows    rows of the output buffers (>= M); sum(m) must not exceed it
+ *   offsets     device int64[G+1], written
+ *   status      device int32, overwritten with the GL_DEV_* flags (0 = ok)
+ * Errors: GL_ERR_INVALID for null pointers, G out of range, negative sizes.
+ */
+gl_status gl_offsets(const int64_t* m_splits, int G, int64_t expect_rows, int64_t out_rows,
+                     int64_t* offsets, int32_t* status, void* stream);
+
+/*
+ * gl_fwd -- grouped forward, y_i = x_i W_i^T (+ b_i).
+ *
+ * ``grouped_linear.py`` (ops/basic) GroupedLinear docstring and fuser_forward
+ * ("Perform GEMMs", one output, per-group bias).  The output may be a caller
+ * buffer with more rows than M ("Add optional caller-provided output/grad-input
+ * buffers", PR #3161): only the packed valid rows [0, M) that belong to a group
+ * are written; rows [M, y_rows) are left untouched.
+ *
+ *   x        device bf16 [M, K]
+ *   w        bf16 weights, [G, N, K] stacked or G pointers to [N, K]
+ *   bias     NULL (no bias) or bf16 [G, N] stacked / G pointers to [N]
+ *   offsets  device int64[G+1] from gl_offsets
+ *   status   device int32 status word from gl_offsets (read; may get TIMEOUT)
+ *   y        device bf16 [y_rows, N], y_rows >= M
+ * Limits: K % 8 == 0, N % 8 == 0 (16-byte row pitch), G <= GL_MAX_GROUPS.
+ * The bias is added to the fp32 accumulator, then one round-to-nearest-even
+ * conversion gives the bf16 output.
+ */
+gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int64_t* offsets,
+                 int32_t* status, int G, int64_t M, int N, int K, void* y, int64_t y_rows,
+                 void* stream);
+
+/*
+ * gl_dgrad -- grouped data gradient, dx_i = dy_i W_i.
+ *
+ * ``grouped_linear.py`` fuser_backward, "Perform dgrad GEMMs" (layout "NN",
+ * one output).  Same caller-buffer rule as gl_fwd: rows [M, dx_rows) are not
+ * written.
+ *
+ *   dy       device bf16 [M, N]
+ *   w        bf16 weights as in gl_fwd
+ *   dx       device bf16 [dx_rows, K], dx_rows >= M
+ * Limits: K % 8 == 0, N % 8 == 0.
+ */
+gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t* status, int G,
+                   int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream);
+
+/*
+ * gl_wgrad -- grouped weight gradient into fp32 main_grad.
+ *
+ * ``grouped_linear.py`` fuser_backward, "Initialize grad weight buffers" and
+ * "Perform wgrad GEMMs" (layout "NT"): dW_i = dy_i^T x_i.  With
+ * accumulate != 0 it is added to main_grad (Megatron-style wgrad fusion);
+ * with accumulate == 0 it overwrites main_grad (``overwrite_main_grad``), so
+ * an empty group gets zeros.  With accumulate != 0 an empty group's
+ * main_grad is not touched.
+ *
+ *   x, dy      device bf16 [M, K] and [M, N]
+ *   main_grad  fp32 [G, N, K] stacked or G pointers to [N, K]
+ * Limits: K % 8 == 0, N % 8 == 0.
+ */
+gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_t* status, int G,
+                   int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream);
+
+/*
+ * group_quantize_mxfp8 -- MXFP8 (E4M3 codes, E8M0 block scales) cast of a
+ * bf16 [rows, cols] tensor whose rows form G groups.
+ *
+ * ``grouped_linear.py`` (ops/basic): MXFP8 tensors hold E4M3 data and one
+ * power-of-two scale per 32 elements, in a rowwise and a columnwise copy
+ * (``_quantize_weights_mxfp8``); inputs and output gradients are quantized
+ * per split (``split_quantize``); the grouped cast kernel is
+ * ``group_quantize_mxfp8`` ("Improve device-init grouped linear module",
+ * PR #3224).  For every block of 32 elements: amax = max |v|; the scale is
+ * 2^e with e the smallest integer such that amax <= 448 * 2^e (clamped to
+ * [-127, 127]; e = 0 when amax = 0), stored as the byte e + 127; each code is
+ * v * 2^-e rounded to the nearest E4M3 value (ties to even, saturating).
+ *
+ *   src         device bf16 [rows, cols]
+ *   row_offsets device int64[G+1] group row offsets, or NULL for G equal
+ *               groups of rows/G rows (a stacked [G, rows/G, cols] weight)
+ *   status      device int32 status word or NULL; non-zero -> nothing written
+ *   codes_r     NULL or device u8 [rows, cols]: rowwise codes (blocks of 32
+ *               along each row)
+ *   scales_r    device u8 [rows, cols/32] (required with codes_r)
+ *   codes_c     NULL or device u8 [rows, cols]: columnwise codes (blocks of 32
+ *               rows along each column, restarting at every group's first
+ *               row; a group's last block may be partial)
+ *   scales_c    device u8 [S, cols] (required with codes_c), where group i's
+ *               block j is scale row sum_{l<i} ceil(m_l/32) + j;
+ *               S <= ceil(rows/32) + G bounds the rows used.
+ * Limits: cols % 32 == 0; rows/G integral when row_offsets is NULL.
+ */
+gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
+                               int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                               uint8_t* codes_c, uint8_t* scales_c, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GL_H_ */

@@ -409,3 +409,26 @@ def rel_frobenius(got: np.ndarray, ref: np.ndarray) -> float:
     if den == 0.0:
         return 0.0 if num == 0.0 else float("inf")
     return float(num / den)
+
+
+# ---------------------------------------------------------------------------
+# Single output entries (for checking full-size runs on a sample)
+# ---------------------------------------------------------------------------
+
+
+def fwd_entry(x_row: np.ndarray, w_row: np.ndarray, b: Optional[float]) -> float:
+    """y[r, n] = sum_k x[r, k] W_g[n, k] (+ b_g[n]) for one (r, n)."""
+    v = float(np.dot(np.asarray(x_row, np.float64), np.asarray(w_row, np.float64)))
+    return v + (0.0 if b is None else float(b))
+
+
+def dgrad_entry(dy_row: np.ndarray, w_col: np.ndarray) -> float:
+    """dx[r, k] = sum_n dy[r, n] W_g[n, k] for one (r, k)."""
+    return float(np.dot(np.asarray(dy_row, np.float64), np.asarray(w_col, np.float64)))
+
+
+def wgrad_entry(dy_col: np.ndarray, x_col: np.ndarray, old: float, accumulate: bool) -> float:
+    """main_grad_g[n, k] (+)= sum_{r in g} dy[r, n] x[r, k] for one (g, n, k);
+    ``dy_col`` / ``x_col`` hold the group's rows only."""
+    v = float(np.dot(np.asarray(dy_col, np.float64), np.asarray(x_col, np.float64)))
+    return (float(old) if accumulate else 0.0) + v

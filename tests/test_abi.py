@@ -1,0 +1,67 @@
+"""The C-ABI library builds, loads and exports every entry point declared in
+include/gl.h; host-side argument checks answer without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from grouped_gemm_splits_b200 import gl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "gl.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:gl_status|int|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = gl.load()
+    names = _declared()
+    assert "gl_fwd" in names and "group_quantize_mxfp8" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(gl.EXPORTED) <= set(names)
+
+
+def test_version_and_status_strings():
+    lib = gl.load()
+    assert lib.gl_version() >= 100
+    assert lib.gl_status_string(gl.GL_ERR_INVALID) == b"invalid argument"
+
+
+def test_host_side_validation_without_gpu():
+    """Invalid arguments are rejected before any CUDA call is made."""
+    lib = gl.load()
+    w = gl.GlGrouped(gl.GL_STACKED, 16, None)
+    # G <= 0, N/K <= 0: ValueError analogues of GroupedLinear's constructor checks
+    assert lib.gl_fwd(16, w, None, 16, 16, 0, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
+    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 0, 8, 16, 8, None) == gl.GL_ERR_INVALID
+    # N % 8 != 0: unsupported row pitch
+    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 12, 8, 16, 8, None) == gl.GL_ERR_UNSUPPORTED
+    # caller buffer with fewer rows than the input
+    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 8, 8, 16, 7, None) == gl.GL_ERR_INVALID
+    # null pointers
+    assert lib.gl_fwd(None, w, None, 16, 16, 2, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
+    assert lib.gl_dgrad(16, w, 16, None, 2, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
+    assert lib.gl_wgrad(16, 16, 16, 16, 2, 8, 8, 8, gl.GlGrouped(gl.GL_STACKED, None, None), 1, None) == gl.GL_ERR_INVALID
+    assert lib.gl_offsets(None, 4, 8, 8, 16, 16, None) == gl.GL_ERR_INVALID
+    assert lib.gl_offsets(16, 0, 8, 8, 16, 16, None) == gl.GL_ERR_INVALID
+    # per-group mode with a null member pointer
+    arr = (ctypes.c_void_p * 2)(16, None)
+    pg = gl.GlGrouped(gl.GL_PER_GROUP, None, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
+    assert lib.gl_fwd(16, pg, None, 16, 16, 2, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
+    # quantize: cols not a multiple of 32; no output requested
+    assert lib.group_quantize_mxfp8(16, 8, 48, None, 1, None, 16, 16, None, None, None) == gl.GL_ERR_UNSUPPORTED
+    assert lib.group_quantize_mxfp8(16, 8, 64, None, 1, None, None, None, None, None, None) == gl.GL_ERR_INVALID
+    assert lib.group_quantize_mxfp8(16, 9, 64, None, 2, None, 16, 16, None, None, None) == gl.GL_ERR_INVALID
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(gl, "_lib", None)
+    monkeypatch.setattr(gl, "_LIB_PATH", str(tmp_path / "libgl.so"))
+    with pytest.raises(gl.GlError):
+        gl.load()
