@@ -69,11 +69,13 @@ gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int6
                  void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  if (x == nullptr || y == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if ((x == nullptr && M > 0) || (y == nullptr && M > 0) || offsets == nullptr || status == nullptr)
+    return GL_ERR_INVALID;
   if (!grouped_ok(w, G) || (bias != nullptr && !grouped_ok(*bias, G))) return GL_ERR_INVALID;
   if (y_rows < M) return GL_ERR_INVALID;
   if (!aligned16(x) || !aligned16(y) || !grouped_aligned(w, G) || (bias && !grouped_aligned(*bias, G)))
     return GL_ERR_UNSUPPORTED;
+  if (M == 0) return GL_OK;  // no rows: nothing to write
   GemmCall c{};
   c.mode = gl::kFwd;
   c.a = x;
@@ -95,10 +97,12 @@ gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t
                    int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  if (dy == nullptr || dx == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if ((dy == nullptr && M > 0) || (dx == nullptr && M > 0) || offsets == nullptr || status == nullptr)
+    return GL_ERR_INVALID;
   if (!grouped_ok(w, G)) return GL_ERR_INVALID;
   if (dx_rows < M) return GL_ERR_INVALID;
   if (!aligned16(dy) || !aligned16(dx) || !grouped_aligned(w, G)) return GL_ERR_UNSUPPORTED;
+  if (M == 0) return GL_OK;
   GemmCall c{};
   c.mode = gl::kDgrad;
   c.a = dy;
@@ -119,9 +123,18 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
                    int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  if (x == nullptr || dy == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if ((x == nullptr && M > 0) || (dy == nullptr && M > 0) || offsets == nullptr || status == nullptr)
+    return GL_ERR_INVALID;
   if (!grouped_ok(main_grad, G)) return GL_ERR_INVALID;
   if (!aligned16(x) || !aligned16(dy) || !grouped_aligned(main_grad, G)) return GL_ERR_UNSUPPORTED;
+  if (M == 0) {
+    if (accumulate) return GL_OK;  // every group is empty: main_grad unchanged
+    // overwrite: the kernel writes zeros and never reads x / dy; give the
+    // operand maps any valid base
+    const void* any = main_grad.mode == GL_STACKED ? main_grad.base : main_grad.ptrs[0];
+    x = any;
+    dy = any;
+  }
   GemmCall c{};
   c.mode = gl::kWgrad;
   c.a = dy;

@@ -16,6 +16,9 @@
  *    [o[i], o[i+1]) of x, y, dy and dx, where o = offsets from gl_offsets.
  *  - Floating types: x, W, b, dy, y, dx are bf16 (2 bytes); main_grad is
  *    fp32.  Products accumulate in fp32 on the tensor cores.
+ *  - When M == 0 (every group empty) the row operands (x, dy, y, dx) may
+ *    be NULL; gl_fwd / gl_dgrad then do nothing and gl_wgrad only zeroes
+ *    main_grad when it overwrites.
  *  - Every call is asynchronous on ``stream`` (a cudaStream_t; NULL is the
  *    legacy default stream) and never synchronises the host: split sizes stay
  *    on the device.
