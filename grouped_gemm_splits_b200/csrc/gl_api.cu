@@ -1,8 +1,12 @@
 // gl_api.cu -- the C ABI (include/gl.h): argument checks, then launches.
 // Nothing here allocates device memory or synchronises the host.
+#include <atomic>
+
 #include "gl_internal.h"
 
 namespace {
+
+std::atomic<int> g_cta_pair{1};
 
 using gl::GemmCall;
 
@@ -57,6 +61,11 @@ const char* gl_status_string(gl_status s) {
   return "unknown status";
 }
 
+gl_status gl_set_cta_pair(int enable) {
+  g_cta_pair.store(enable ? 1 : 0);
+  return GL_OK;
+}
+
 gl_status gl_offsets(const int64_t* m_splits, int G, int64_t expect_rows, int64_t out_rows,
                      int64_t* offsets, int32_t* status, void* stream) {
   if (m_splits == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
@@ -89,6 +98,7 @@ gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int6
   c.M = M;
   c.N = N;
   c.K = K;
+  c.cta_pair = g_cta_pair.load();
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -115,6 +125,7 @@ gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t
   c.M = M;
   c.N = N;
   c.K = K;
+  c.cta_pair = g_cta_pair.load();
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -147,6 +158,7 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
   c.N = N;
   c.K = K;
   c.accumulate = accumulate ? 1 : 0;
+  c.cta_pair = g_cta_pair.load();
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }

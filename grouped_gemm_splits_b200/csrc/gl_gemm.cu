@@ -4,19 +4,32 @@
 // (TransformerEngine ``grouped_linear.py``, ops/basic: fuser_forward "Perform
 // GEMMs" and fuser_backward "Perform dgrad GEMMs" / "Perform wgrad GEMMs"):
 //
-//   FWD    y[r, n]        = sum_k x[r, k]  W_g[n, k]   (+ b_g[n])   rows r of group g
-//   DGRAD  dx[r, k]       = sum_n dy[r, n] W_g[n, k]                rows r of group g
+//   FWD    y[r, n]          = sum_k x[r, k]  W_g[n, k]   (+ b_g[n])   rows r of group g
+//   DGRAD  dx[r, k]         = sum_n dy[r, n] W_g[n, k]                rows r of group g
 //   WGRAD  main_grad_g[n,k] (+)= sum_{r in g} dy[r, n] x[r, k]
 //
-// Each CTA owns one SM.  Warp 0 streams operand tiles with TMA into a ring of
-// shared-memory stages, warp 1 issues tcgen05.mma (fp32 accumulators in
-// TMEM, two 128x256 accumulators so the epilogue of one tile overlaps the
-// main loop of the next) and warps 2-5 drain TMEM: bias + bf16 rounding and
-// row-clipped stores for FWD/DGRAD, TMA reduce-add (accumulate) or TMA store
-// (overwrite) of fp32 main_grad tiles for WGRAD.  Tiles are enumerated group
-// by group from the device offsets (a tile prefix built in shared memory), so
-// empty groups cost nothing and the host never learns the split sizes.
+// Persistent kernel, one CTA per SM.  With CG = 2 the CTAs of a cluster pair
+// compute one 256 x 256 accumulator tile with tcgen05.mma.cta_group::2: each
+// CTA streams its own 128 rows of A and its own half of B (no multicast
+// loads), the peer CTA relays "stage landed" to the leader with a remote
+// mbarrier arrive, the leader issues the MMAs and its tcgen05.commit
+// multicasts stage-free / accumulator-full to both CTAs.  With CG = 1 a CTA
+// computes a 128 x 256 tile alone.
+//
+// Roles: warp 0 TMA producer (128-byte swizzled boxes into a ring of
+// shared-memory stages), warp 1 TMEM owner and MMA issuer (leader) or stage
+// relay (peer), warps 2-5 epilogue (TMEM -> registers; bias + bf16 rounding
+// and row-clipped stores for FWD/DGRAD; TMA reduce-add or TMA store of fp32
+// main_grad boxes for WGRAD).  Two accumulators in TMEM let a tile's
+// epilogue overlap the next tile's main loop.  Tiles are enumerated group by
+// group from the device offsets (tile prefix in shared memory): empty groups
+// cost nothing and the host never learns the split sizes.
 #include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "gl_internal.h"
 #include "gl_ptx.cuh"
@@ -24,31 +37,35 @@
 namespace gl {
 namespace {
 
-constexpr int BM = 128;  // accumulator rows (TMEM lanes)
-constexpr int BN = 256;  // accumulator columns
-constexpr int BK = 64;   // contraction elements per stage (one 128-byte swizzle row)
+constexpr int BK = 64;  // contraction elements per stage (one 128-byte swizzle row)
 constexpr int kThreads = 192;
 constexpr int kPG = 64;  // per-group tensor maps carried by one launch
+constexpr int kSmemBudget = 196608;
 
-template <int MODE>
+template <int MODE, int CG>
 struct Cfg {
-  static constexpr int kStages = (MODE == kWgrad) ? 3 : 4;
-  static constexpr int kABytes = BM * BK * 2;  // 16 KB
-  static constexpr int kBBytes = BN * BK * 2;  // 32 KB
+  static constexpr int kTileM = 128 * CG;          // accumulator rows per tile (pair)
+  static constexpr int kTileN = 256;               // accumulator columns
+  static constexpr int kBRows = kTileN / CG;       // rows of the B operand held per CTA
+  static constexpr int kABytes = 128 * BK * 2;     // 16 KB
+  static constexpr int kBBytes = kBRows * BK * 2;  // 32 KB (CG 1) or 16 KB (CG 2)
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStagingBytes = (MODE == kWgrad) ? 2 * BM * 32 * 4 : 0;  // 2 x 16 KB
+  static constexpr int kStagingBytes = (MODE == kWgrad) ? 2 * 128 * 32 * 4 : 0;  // 2 x 16 KB
+  static constexpr int kStages = (kSmemBudget - kStagingBytes) / kStageBytes;
   static constexpr int kBarOffset = kStages * kStageBytes + kStagingBytes;
   static constexpr int kBarBytes = 256;
   static constexpr int kPrefixOffset = kBarOffset + kBarBytes;
-  // A / B operand storage in shared memory: 1 = MN-major (see file header)
+  // shared-memory majorness of the operands (1 = MN-major)
   static constexpr int kAMN = (MODE == kWgrad) ? 1 : 0;
   static constexpr int kBMN = (MODE == kFwd) ? 0 : 1;
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, kAMN, kBMN);
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kTileN, kAMN, kBMN);
+  static_assert(kStages >= 3, "pipeline too shallow");
+  static_assert(kBarOffset % 1024 == 0, "stage alignment");
 };
 
 struct GemmParams {
   CUtensorMap tmA;    // FWD x{K,M} box{64,128}; DGRAD dy{N,M} box{64,128}; WGRAD dy{N,M} box{64,64}
-  CUtensorMap tmB;    // stacked W{K,N,G}: FWD box{64,256,1}, DGRAD box{64,64,1}; WGRAD x{K,M} box{64,64}
+  CUtensorMap tmB;    // stacked W{K,N,G}: FWD box{64,BRows,1}, DGRAD box{64,64,1}; WGRAD x{K,M} box{64,64}
   CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,128,1}
   const int64_t* offsets;  // G+1 entries
   int32_t* status;
@@ -80,22 +97,24 @@ struct Tile {
   int g;
   int num_kb;
   int mt, nt;
-  int64_t r0, r1;  // FWD/DGRAD: output rows [r0, r1) clip; WGRAD: contraction rows [r0, r1)
+  int64_t r0, r1;  // FWD/DGRAD: tile's first row, group end; WGRAD: contraction rows [r0, r1)
 };
 
 __device__ __forceinline__ int ceil_div_i(int64_t a, int b) { return static_cast<int>((a + b - 1) / b); }
 
-template <int MODE>
+template <int MODE, int CG>
 __device__ __forceinline__ int tiles_of_group(int64_t m, const GemmParams& p) {
-  if (MODE == kFwd) return m > 0 ? ceil_div_i(m, BM) * ceil_div_i(p.N, BN) : 0;
-  if (MODE == kDgrad) return m > 0 ? ceil_div_i(m, BM) * ceil_div_i(p.K, BN) : 0;
-  return (m > 0 || !p.accumulate) ? ceil_div_i(p.N, BM) * ceil_div_i(p.K, BN) : 0;
+  using C = Cfg<MODE, CG>;
+  if (MODE == kFwd) return m > 0 ? ceil_div_i(m, C::kTileM) * ceil_div_i(p.N, C::kTileN) : 0;
+  if (MODE == kDgrad) return m > 0 ? ceil_div_i(m, C::kTileM) * ceil_div_i(p.K, C::kTileN) : 0;
+  return (m > 0 || !p.accumulate) ? ceil_div_i(p.N, C::kTileM) * ceil_div_i(p.K, C::kTileN) : 0;
 }
 
-template <int MODE>
+template <int MODE, int CG>
 __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const GemmParams& p) {
+  using C = Cfg<MODE, CG>;
   // largest g with prefix[g] <= t (prefix is non-decreasing, prefix[0] = 0)
-  int lo = 0, hi = p.G;  // answer in [lo, hi)
+  int lo = 0, hi = p.G;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (prefix[mid] <= t) lo = mid; else hi = mid;
@@ -106,17 +125,17 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const Gemm
   const int64_t o0 = __ldg(p.offsets + lo), o1 = __ldg(p.offsets + lo + 1);
   const int64_t m = o1 > o0 ? o1 - o0 : 0;
   if (MODE == kWgrad) {
-    const int mtn = ceil_div_i(p.N, BM);
+    const int mtn = ceil_div_i(p.N, C::kTileM);
     tl.mt = local % mtn;
     tl.nt = local / mtn;
     tl.r0 = o0;
     tl.r1 = o0 + m;
     tl.num_kb = ceil_div_i(m, BK);
   } else {
-    const int mtg = ceil_div_i(m, BM);
+    const int mtg = ceil_div_i(m, C::kTileM);
     tl.mt = local % mtg;  // m-tiles fastest: neighbouring CTAs share a weight strip
     tl.nt = local / mtg;
-    tl.r0 = o0 + static_cast<int64_t>(tl.mt) * BM;
+    tl.r0 = o0 + static_cast<int64_t>(tl.mt) * C::kTileM;
     tl.r1 = o0 + m;
     tl.num_kb = ceil_div_i(MODE == kFwd ? p.K : p.N, BK);
   }
@@ -135,10 +154,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int MODE, bool PG>
+// Zero rows [r_from, r_to) of this CTA's A and B stage buffers (MN-major, 64
+// rows x 128 bytes per 8 KB chunk) so rows past a group's end add nothing to
+// a wgrad contraction.  Executed by one full warp.
+template <int MODE, int CG>
+__device__ __forceinline__ void zero_tail_rows(uint8_t* sa, uint8_t* sb, int r_from, int r_to, int lane) {
+  using C = Cfg<MODE, CG>;
+  constexpr int kChunksA = 2, kChunksB = C::kBRows / 64;
+  const int nrows = r_to - r_from;
+  if (nrows <= 0) return;
+  const int per_chunk = nrows * 8;  // 16-byte pieces per chunk
+  for (int idx = lane; idx < (kChunksA + kChunksB) * per_chunk; idx += 32) {
+    const int chunk = idx / per_chunk;
+    const int rem = idx - chunk * per_chunk;
+    const int row = r_from + (rem >> 3);
+    uint8_t* base = (chunk < kChunksA) ? (sa + chunk * 8192) : (sb + (chunk - kChunksA) * 8192);
+    *reinterpret_cast<uint4*>(base + row * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+}
+
+template <int MODE, int CG, bool PG>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ PGArgs<PG> pg) {
-  using C = Cfg<MODE>;
+  using C = Cfg<MODE, CG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -153,23 +192,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
 
   if (threadIdx.x == 0) {
     *skip_flag = (p.status != nullptr && *reinterpret_cast<volatile int32_t*>(p.status) != 0) ? 1 : 0;
     *abort_flag = 0;
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], (CG == 2 && leader) ? 2 : 1);  // leader: own TMA + peer's relay
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[b], 4 * CG);  // one arrival per epilogue warp of the pair
     }
     mbar_init(mma_done, 1);
     fence_barrier_init();
   }
-  __syncthreads();
-  if (*skip_flag) return;  // bad split sizes reported by gl_offsets: write nothing
+  bool skip;
+  if (CG == 2) {
+    cluster_sync();  // barriers of both CTAs initialised; both skip flags written
+    uint32_t peer_skip;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];"
+                 : "=r"(peer_skip)
+                 : "r"(mapa_shared(smem_u32(const_cast<int*>(skip_flag)), rank ^ 1u))
+                 : "memory");
+    skip = (*skip_flag != 0) || (peer_skip != 0);
+    cluster_sync();  // nobody leaves before the peer has read its flag
+  } else {
+    __syncthreads();
+    skip = *skip_flag != 0;
+  }
+  if (skip) return;  // bad split sizes reported by gl_offsets: write nothing
+
+  const int pair = (CG == 2) ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int npairs = (CG == 2) ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     // tile prefix over groups: prefix[g] = number of tiles of groups < g
@@ -179,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int cnt = 0;
       if (i < p.G) {
         const int64_t m = __ldg(p.offsets + i + 1) - __ldg(p.offsets + i);
-        cnt = tiles_of_group<MODE>(m, p);
+        cnt = tiles_of_group<MODE, CG>(m, p);
       }
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -191,57 +248,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) prefix[0] = 0;
   } else if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * BN);  // two 128 x 256 fp32 accumulators = all 512 columns
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(tmem_slot, 512);  // two 128 x 256 fp32 accumulators per CTA
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 512);
+      tmem_relinquish();
+    }
   } else if (warp == 2 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
-    if (!PG) tma_prefetch_desc(&p.tmB);
-    if (MODE == kWgrad) tma_prefetch_desc(PG ? pg.map(0) : &p.tmOut);
+    if (!PG || MODE == kWgrad) tma_prefetch_desc(&p.tmB);
+    if (MODE == kWgrad && !PG) tma_prefetch_desc(&p.tmOut);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = prefix[p.G];
+  const int hr = static_cast<int>(rank) * 128;        // this CTA's A rows within the tile
+  const int hb = static_cast<int>(rank) * C::kBRows;  // this CTA's B rows within the tile
 
   if (warp == 0) {
-    // ===================== TMA producer =====================
+    // ===================== TMA producer (both CTAs) =====================
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-        const Tile tl = decode_tile<MODE>(t, prefix, p);
+      for (int t = pair; t < total && !*abort_flag; t += npairs) {
+        const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
         for (int kb = 0; kb < tl.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { report_abort(abort_flag, p.status); break; }
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
           if (MODE == kFwd) {
-            tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0));
-            if (PG) tma_load_2d(sb, pg.map(tl.g), &full[stage], kb * BK, tl.nt * BN);
-            else    tma_load_3d(sb, &p.tmB, &full[stage], kb * BK, tl.nt * BN, tl.g);
+            const int n0 = tl.nt * C::kTileN + hb;
+            tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0 + hr));
+            if (PG) tma_load_2d(sb, pg.map(tl.g), &full[stage], kb * BK, n0);
+            else    tma_load_3d(sb, &p.tmB, &full[stage], kb * BK, n0, tl.g);
           } else if (MODE == kDgrad) {
-            tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0));
+            const int n0 = tl.nt * C::kTileN + hb;
+            tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0 + hr));
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c) {
-              if (PG) tma_load_2d(sb + c * 8192, pg.map(tl.g), &full[stage], tl.nt * BN + c * 64, kb * BK);
-              else    tma_load_3d(sb + c * 8192, &p.tmB, &full[stage], tl.nt * BN + c * 64, kb * BK, tl.g);
+            for (int c = 0; c < C::kBRows / 64; ++c) {
+              if (PG) tma_load_2d(sb + c * 8192, pg.map(tl.g), &full[stage], n0 + c * 64, kb * BK);
+              else    tma_load_3d(sb + c * 8192, &p.tmB, &full[stage], n0 + c * 64, kb * BK, tl.g);
             }
           } else {
             const int32_t row = static_cast<int32_t>(tl.r0 + kb * BK);
+            const int m0 = tl.mt * C::kTileM + hr;
+            const int n0 = tl.nt * C::kTileN + hb;
 #pragma unroll
-            for (int c = 0; c < BM / 64; ++c)
-              tma_load_2d(sa + c * 8192, &p.tmA, &full[stage], tl.mt * BM + c * 64, row);
+            for (int c = 0; c < 2; ++c) tma_load_2d(sa + c * 8192, &p.tmA, &full[stage], m0 + c * 64, row);
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_2d(sb + c * 8192, &p.tmB, &full[stage], tl.nt * BN + c * 64, row);
+            for (int c = 0; c < C::kBRows / 64; ++c)
+              tma_load_2d(sb + c * 8192, &p.tmB, &full[stage], n0 + c * 64, row);
           }
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      // Do not leave while a TMA load may still be writing shared memory.
+      // Do not leave while a TMA load may still be writing shared memory: wait
+      // (bounded) for the last stages this thread filled.
       const int inflight = issued < C::kStages ? issued : C::kStages;
       int s = stage;
       uint32_t ph = phase;
@@ -251,92 +319,117 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ===================== MMA issuer =====================
-    int stage = 0;
-    uint32_t phase = 0;
-    int it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const Tile tl = decode_tile<MODE>(t, prefix, p);
-      const int buf = it & 1;
-      const uint32_t tph = (it >> 1) & 1;
-      // every lane waits; the warp acts on a unanimous result
-      if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], tph ^ 1u, abort_flag))) {
-        report_abort(abort_flag, p.status);
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + buf * BN;
-      bool ok = true;
-      for (int kb = 0; kb < tl.num_kb; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+    if (leader) {
+      // ===================== MMA issuer =====================
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int t = pair; t < total; t += npairs, ++it) {
+        const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
+        const int buf = it & 1;
+        const uint32_t tph = (it >> 1) & 1;
+        // every lane waits; the warp acts on a unanimous result
+        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], tph ^ 1u, abort_flag))) {
           report_abort(abort_flag, p.status);
-          ok = false;
           break;
         }
         tc_fence_after();
-        uint8_t* sa = smem + stage * C::kStageBytes;
-        uint8_t* sb = sa + C::kABytes;
-        int ksteps = BK / 16;
-        if (MODE == kWgrad && kb == tl.num_kb - 1) {
-          // Ragged contraction: rows past the group's end must not contribute.
-          // Skip whole 16-row MMA steps beyond the end and zero the rows of the
-          // last partial step in both operands.
-          const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
-          if (valid < BK) {
-            ksteps = (valid + 15) >> 4;
-            const int zend = ksteps * 16;
-            const int nrows = zend - valid;
-            if (nrows > 0) {
-              // 6 chunks (2 of A, 4 of B) of [64 rows x 128 B]; 8 x 16 B per row
-              const int per_chunk = nrows * 8;
-              for (int idx = lane; idx < 6 * per_chunk; idx += 32) {
-                const int chunk = idx / per_chunk;
-                const int rem = idx - chunk * per_chunk;
-                const int row = valid + (rem >> 3);
-                uint8_t* base = (chunk < 2) ? (sa + chunk * 8192) : (sb + (chunk - 2) * 8192);
-                *reinterpret_cast<uint4*>(base + row * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
-              }
-              fence_proxy_async_smem();
+        const uint32_t d_tmem = tmem_base + buf * C::kTileN;
+        bool ok = true;
+        for (int kb = 0; kb < tl.num_kb; ++kb) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+            report_abort(abort_flag, p.status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* sa = smem + stage * C::kStageBytes;
+          uint8_t* sb = sa + C::kABytes;
+          int ksteps = BK / 16;
+          if (MODE == kWgrad && kb == tl.num_kb - 1) {
+            // Ragged contraction: skip whole 16-row MMA steps past the group's
+            // end and zero the rows of the last partial step.
+            const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
+            if (valid < BK) {
+              ksteps = (valid + 15) >> 4;
+              zero_tail_rows<MODE, CG>(sa, sb, valid, ksteps * 16, lane);
             }
           }
-        }
-        __syncwarp();
-        if (lane == 0) {
-          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
-          for (int ks = 0; ks < ksteps; ++ks) {
-            uint64_t ad, bd;
-            if (C::kAMN) ad = smem_desc_sw128(a0 + ks * 2048, 8192, 1024);
-            else         ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
-            if (C::kBMN) bd = smem_desc_sw128(b0 + ks * 2048, 8192, 1024);
-            else         bd = smem_desc_sw128(b0 + ks * 32, 16, 1024);
-            mma_bf16_ss(d_tmem, ad, bd, C::kIdesc, (kb > 0 || ks > 0) ? 1u : 0u);
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
+            for (int ks = 0; ks < ksteps; ++ks) {
+              const uint64_t ad = C::kAMN ? smem_desc_sw128(a0 + ks * 2048, 8192, 1024)
+                                          : smem_desc_sw128(a0 + ks * 32, 16, 1024);
+              const uint64_t bd = C::kBMN ? smem_desc_sw128(b0 + ks * 2048, 8192, 1024)
+                                          : smem_desc_sw128(b0 + ks * 32, 16, 1024);
+              const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+              if (CG == 2) mma_bf16_ss_pair(d_tmem, ad, bd, C::kIdesc, acc);
+              else         mma_bf16_ss(d_tmem, ad, bd, C::kIdesc, acc);
+            }
+            // free the stage (in both CTAs) once these MMAs have read it
+            if (CG == 2) tc_commit_pair_mc(&empty[stage], 0x3);
+            else         tc_commit(&empty[stage]);
           }
-          tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          __syncwarp();
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          if (tl.num_kb > 0) {
+            if (CG == 2) tc_commit_pair_mc(&tfull[buf], 0x3);
+            else         tc_commit(&tfull[buf]);
+          } else {
+            // nothing accumulated: the epilogues write zeros
+            mbar_arrive(&tfull[buf]);
+            if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&tfull[buf]), 1));
+          }
         }
         __syncwarp();
-        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
       }
-      if (!ok) break;
       if (lane == 0) {
-        if (tl.num_kb > 0) tc_commit(&tfull[buf]);
-        else mbar_arrive(&tfull[buf]);  // nothing accumulated: epilogue writes zeros
+        if (CG == 2) tc_commit_pair_mc(mma_done, 0x1);
+        else         tc_commit(mma_done);
+        mbar_wait_bounded(mma_done, 0);  // no MMA in flight past this point
       }
       __syncwarp();
+    } else {
+      // ===================== peer: stage relay =====================
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = pair; t < total; t += npairs) {
+        const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
+        bool ok = true;
+        for (int kb = 0; kb < tl.num_kb; ++kb) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+            report_abort(abort_flag, p.status);
+            ok = false;
+            break;
+          }
+          if (MODE == kWgrad && kb == tl.num_kb - 1) {
+            const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
+            if (valid < BK) {
+              uint8_t* sa = smem + stage * C::kStageBytes;
+              zero_tail_rows<MODE, CG>(sa, sa + C::kABytes, valid, ((valid + 15) >> 4) * 16, lane);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&full[stage]), 0));
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
     }
-    if (lane == 0) {
-      tc_commit(mma_done);  // all MMAs issued by this thread have completed
-      mbar_wait_bounded(mma_done, 0);
-    }
-    __syncwarp();
   } else {
-    // ===================== epilogue (warps 2..5) =====================
+    // ===================== epilogue (warps 2..5, both CTAs) =====================
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
     const bool issuer = (warp == 2 && lane == 0);
+    const uint32_t tempty_leader = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : 0u;
     int it = 0;
     int chunk_ctr = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const Tile tl = decode_tile<MODE>(t, prefix, p);
+    for (int t = pair; t < total; t += npairs, ++it) {
+      const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
       const int buf = it & 1;
       const uint32_t tph = (it >> 1) & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
@@ -356,28 +449,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t tacc = tmem_base + buf * BN + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t tacc = tmem_base + buf * C::kTileN + (static_cast<uint32_t>(q * 32) << 16);
+      auto release_acc = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 2) mbar_arrive_cluster(tempty_leader + buf * 8);
+          else         mbar_arrive(&tempty[buf]);
+        }
+      };
 
       if (MODE != kWgrad) {
         const int Nout = (MODE == kFwd) ? p.N : p.K;
-        const int64_t row = tl.r0 + row_in_tile;
+        const int64_t row = tl.r0 + hr + row_in_tile;
         const bool row_ok = row >= 0 && row < tl.r1 && row < p.out_rows;
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
         const __nv_bfloat16* bias = nullptr;
         if (MODE == kFwd && p.has_bias)
           bias = PG ? pg.b(tl.g) : (p.bias + static_cast<int64_t>(tl.g) * p.N);
-        const int nchunks = min(BN / 32, ceil_div_i(Nout - tl.nt * BN, 32));
+        const int nchunks = min(C::kTileN / 32, ceil_div_i(Nout - tl.nt * C::kTileN, 32));
         for (int c = 0; c < nchunks; ++c) {
-          const int n = tl.nt * BN + c * 32;
+          const int n = tl.nt * C::kTileN + c * 32;
           uint32_t r[32];
           tmem_ld_32x32b_x32(tacc + c * 32, r);
           tmem_ld_wait();
-          if (c == nchunks - 1) {
-            // accumulator fully read: hand the buffer back to the MMA warp
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
-          }
+          if (c == nchunks - 1) release_acc();  // accumulator fully read
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -407,20 +503,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (nchunks <= 0) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
-        }
       } else {
-        // main_grad tile: rows n0.. (TMEM lanes) x cols k0.. (TMEM columns)
+        // main_grad box: rows n0.. (TMEM lanes) x cols k0.. (TMEM columns)
         float* staging = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
-        const int n0 = tl.mt * BM;
-        const int k0 = tl.nt * BN;
-        const int nchunks = min(BN / 32, ceil_div_i(p.K - k0, 32));
+        const int n0 = tl.mt * C::kTileM + hr;
+        const int k0 = tl.nt * C::kTileN;
+        const int nchunks = min(C::kTileN / 32, ceil_div_i(p.K - k0, 32));
         const bool have_acc = tl.num_kb > 0;
+        const bool rows_in = n0 < p.N;  // the pair's second half may lie past N
         for (int c = 0; c < nchunks; ++c, ++chunk_ctr) {
-          float* stg = staging + (chunk_ctr & 1) * (BM * 32);
+          float* stg = staging + (chunk_ctr & 1) * (128 * 32);
           if (issuer) bulk_wait_group_read<1>();  // the buffer's previous store has read it
           named_barrier_sync(1, 128);
           uint32_t r[32];
@@ -431,11 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) r[j] = 0u;
           }
-          if (c == nchunks - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
-          }
+          if (c == nchunks - 1) release_acc();
           // row `row_in_tile` of a [128 x 32] fp32 box, 128-byte swizzle
           uint8_t* rowp = reinterpret_cast<uint8_t*>(stg) + row_in_tile * 128;
 #pragma unroll
@@ -445,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           named_barrier_sync(1, 128);
-          if (issuer) {
+          if (issuer && rows_in) {
             const int kc = k0 + c * 32;
             if (PG) {
               if (p.accumulate) tma_reduce_add_2d(pg.map(tl.g), stg, kc, n0);
@@ -457,27 +545,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit_group();
           }
         }
-        if (nchunks <= 0) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
-        }
       }
     }
     if (MODE == kWgrad && issuer) bulk_wait_group<0>();
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * BN);
+    if (CG == 2) tmem_dealloc_pair(tmem_base, 512);
+    else         tmem_dealloc(tmem_base, 512);
   }
 }
 
-template <int MODE>
+template <int MODE, int CG>
 constexpr int smem_bytes_for(int G) {
-  return Cfg<MODE>::kPrefixOffset + (G + 1) * 4 + 1024;  // + alignment slack
+  return Cfg<MODE, CG>::kPrefixOffset + (G + 1) * 4 + 1024;  // + alignment slack
 }
 
 bool make_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_in,
@@ -496,17 +580,65 @@ bool make_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uin
   return encode_tmap(m, dt, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int MODE, bool PG>
+cudaLaunchConfig_t pair_config(int grid, int smem, cudaStream_t stream, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Persistent grid: one CTA per SM, or as many CTA pairs as can be resident.
+template <typename Kern>
+int grid_for(Kern kern, int cg, int smem) {
+  if (cg == 1) return num_sms();
+  static std::mutex mu;
+  static std::unordered_map<const void*, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const void* key = reinterpret_cast<const void*>(reinterpret_cast<uintptr_t>(kern) ^ (static_cast<uintptr_t>(dev) << 48));
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config(2 * (num_sms() / 2), smem, nullptr, attr);
+  int nclusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters <= 0)
+    nclusters = num_sms() / 2;
+  const int grid = 2 * std::min(nclusters, num_sms() / 2);
+  std::lock_guard<std::mutex> lk(mu);
+  cache[key] = grid;
+  return grid;
+}
+
+template <int MODE, int CG, bool PG>
 gl_status launch_one(const GemmParams& prm, const PGArgs<PG>& pga, int G, cudaStream_t stream) {
-  const int smem = smem_bytes_for<MODE>(G);
-  auto kern = grouped_gemm_kernel<MODE, PG>;
+  const int smem = smem_bytes_for<MODE, CG>(G);
+  auto kern = grouped_gemm_kernel<MODE, CG, PG>;
   if (set_max_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return GL_ERR_CUDA;
-  kern<<<num_sms(), kThreads, smem, stream>>>(prm, pga);
+  const int grid = grid_for(kern, CG, smem);
+  if (CG == 1) {
+    kern<<<grid, kThreads, smem, stream>>>(prm, pga);
+  } else {
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pair_config(grid, smem, stream, attr);
+    if (cudaLaunchKernelEx(&cfg, kern, prm, pga) != cudaSuccess) return GL_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
 }
 
-template <int MODE>
+template <int MODE, int CG>
 gl_status launch_mode(const GemmCall& c) {
+  using Cf = Cfg<MODE, CG>;
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   GemmParams prm;
   memset(&prm, 0, sizeof(prm));
@@ -521,9 +653,9 @@ gl_status launch_mode(const GemmCall& c) {
   const uint64_t Mrows = c.M > 0 ? static_cast<uint64_t>(c.M) : 1;  // a map needs >= 1 row
   bool ok = true;
   if (MODE == kFwd) {
-    ok &= make_2d(&prm.tmA, c.a, c.K, Mrows, BK, BM, BF, 2);
+    ok &= make_2d(&prm.tmA, c.a, c.K, Mrows, BK, 128, BF, 2);
   } else if (MODE == kDgrad) {
-    ok &= make_2d(&prm.tmA, c.a, c.N, Mrows, BK, BM, BF, 2);
+    ok &= make_2d(&prm.tmA, c.a, c.N, Mrows, BK, 128, BF, 2);
   } else {
     ok &= make_2d(&prm.tmA, c.a, c.N, Mrows, 64, BK, BF, 2);
     ok &= make_2d(&prm.tmB, c.b, c.K, Mrows, 64, BK, BF, 2);
@@ -533,16 +665,16 @@ gl_status launch_mode(const GemmCall& c) {
   const bool stacked = (MODE == kWgrad) ? (c.out_grouped.mode == GL_STACKED) : (c.w.mode == GL_STACKED);
   const bool bias_stacked = prm.has_bias && c.bias->mode == GL_STACKED;
   if (stacked && (!prm.has_bias || bias_stacked)) {
-    if (MODE == kFwd) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, BK, BN, BF, 2);
+    if (MODE == kFwd) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, BK, Cf::kBRows, BF, 2);
     if (MODE == kDgrad) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, 64, BK, BF, 2);
     if (MODE == kWgrad)
-      ok &= make_3d(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 32, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+      ok &= make_3d(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 32, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
     if (!ok) return GL_ERR_UNSUPPORTED;
     prm.offsets = c.offsets;
     prm.G = c.G;
     if (prm.has_bias) prm.bias = reinterpret_cast<const __nv_bfloat16*>(c.bias->base);
     PGArgs<false> none{0};
-    return launch_one<MODE, false>(prm, none, c.G, c.stream);
+    return launch_one<MODE, CG, false>(prm, none, c.G, c.stream);
   }
   // Per-group pointers (weights, biases or main_grad): launches of <= kPG groups.
   PGArgs<true>* pga = new PGArgs<true>;
@@ -556,7 +688,7 @@ gl_status launch_mode(const GemmCall& c) {
         const void* wp = (c.w.mode == GL_STACKED)
                              ? static_cast<const uint8_t*>(c.w.base) + static_cast<size_t>(g) * c.N * c.K * 2
                              : c.w.ptrs[g];
-        if (MODE == kFwd) ok &= make_2d(&pga->tm[i], wp, c.K, c.N, BK, BN, BF, 2);
+        if (MODE == kFwd) ok &= make_2d(&pga->tm[i], wp, c.K, c.N, BK, Cf::kBRows, BF, 2);
         else              ok &= make_2d(&pga->tm[i], wp, c.K, c.N, 64, BK, BF, 2);
         if (prm.has_bias)
           pga->bias[i] = reinterpret_cast<const __nv_bfloat16*>(
@@ -567,25 +699,30 @@ gl_status launch_mode(const GemmCall& c) {
         const void* gp = (c.out_grouped.mode == GL_STACKED)
                              ? static_cast<const uint8_t*>(c.out_grouped.base) + static_cast<size_t>(g) * c.N * c.K * 4
                              : c.out_grouped.ptrs[g];
-        ok &= make_2d(&pga->tm[i], gp, c.K, c.N, 32, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+        ok &= make_2d(&pga->tm[i], gp, c.K, c.N, 32, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
       }
     }
     if (!ok) { st = GL_ERR_UNSUPPORTED; break; }
     prm.offsets = c.offsets + g0;
     prm.G = cg;
-    st = launch_one<MODE, true>(prm, *pga, cg, c.stream);
+    st = launch_one<MODE, CG, true>(prm, *pga, cg, c.stream);
   }
   delete pga;
   return st;
+}
+
+template <int MODE>
+gl_status launch_cg(const GemmCall& c) {
+  return c.cta_pair ? launch_mode<MODE, 2>(c) : launch_mode<MODE, 1>(c);
 }
 
 }  // namespace
 
 gl_status launch_grouped_gemm(const GemmCall& c) {
   switch (c.mode) {
-    case kFwd: return launch_mode<kFwd>(c);
-    case kDgrad: return launch_mode<kDgrad>(c);
-    case kWgrad: return launch_mode<kWgrad>(c);
+    case kFwd: return launch_cg<kFwd>(c);
+    case kDgrad: return launch_cg<kDgrad>(c);
+    case kWgrad: return launch_cg<kWgrad>(c);
   }
   return GL_ERR_INVALID;
 }

@@ -39,6 +39,7 @@ struct GemmCall {
   int64_t M;
   int N, K;
   int accumulate;
+  int cta_pair;  // 1: 256x256 tiles on CTA pairs (cta_group::2); 0: 128x256 tiles per CTA
   cudaStream_t stream;
 };
 

@@ -22,7 +22,7 @@ GL_OK, GL_ERR_INVALID, GL_ERR_UNSUPPORTED, GL_ERR_CUDA = 0, 1, 2, 3
 GL_DEV_NEG_SPLIT, GL_DEV_SUM_MISMATCH, GL_DEV_OUT_OVERFLOW, GL_DEV_TIMEOUT = 1, 2, 4, 8
 GL_STACKED, GL_PER_GROUP = 0, 1
 
-EXPORTED = ("gl_version", "gl_status_string", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
+EXPORTED = ("gl_version", "gl_status_string", "gl_set_cta_pair", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
             "group_quantize_mxfp8")
 
 
@@ -51,6 +51,8 @@ def load() -> ctypes.CDLL:
     L.gl_version.restype = i32
     L.gl_status_string.restype = ctypes.c_char_p
     L.gl_status_string.argtypes = [i32]
+    L.gl_set_cta_pair.restype = i32
+    L.gl_set_cta_pair.argtypes = [i32]
     L.gl_offsets.restype = i32
     L.gl_offsets.argtypes = [vp, i32, i64, i64, vp, vp, vp]
     L.gl_fwd.restype = i32
@@ -96,6 +98,11 @@ def _grouped(t: TensorOrList, G: int):
 
 def _shape_nk(w: TensorOrList):
     return tuple((w if isinstance(w, torch.Tensor) else w[0]).shape[-2:])
+
+
+def gl_set_cta_pair(enable: bool) -> None:
+    """Tile shape of later GEMM launches: CTA pairs (256x256, default) or single CTAs (128x256)."""
+    _check(load().gl_set_cta_pair(1 if enable else 0), "gl_set_cta_pair")
 
 
 def gl_offsets(m_splits: torch.Tensor, expect_rows: int, out_rows: Optional[int] = None,

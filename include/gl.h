@@ -82,6 +82,15 @@ int gl_version(void);
 const char* gl_status_string(gl_status s);
 
 /*
+ * gl_set_cta_pair -- tile shape of the grouped GEMMs launched afterwards by
+ * this process: enable != 0 (the default) computes 256 x 256 output tiles on
+ * pairs of CTAs (tcgen05 cta_group::2, one CTA per SM); enable == 0 computes
+ * 128 x 256 tiles on single CTAs.  Results agree within rounding; the pair
+ * shape moves less operand data per flop.  Always returns GL_OK.
+ */
+gl_status gl_set_cta_pair(int enable);
+
+/*
  * gl_offsets -- group row offsets from the split sizes, on the device.
  *
  * Computes o[0] = 0 and o[i+1] = o[i] + m_splits[i] (int64, G+1 values),

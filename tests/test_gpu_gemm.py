@@ -18,6 +18,15 @@ from tests.gpu_util import (TOL_BF16, assert_groups_close, f64, offsets_on_devic
 
 pytestmark = pytest.mark.gpu
 
+
+@pytest.fixture(params=["pair", "single"])
+def tile_mode(request):
+    """Run a test with 256x256 tiles on CTA pairs and with 128x256 tiles on
+    single CTAs; the default (pairs) is restored afterwards."""
+    gl.gl_set_cta_pair(request.param == "pair")
+    yield request.param
+    gl.gl_set_cta_pair(True)
+
 # (G, N, K, m_splits): several tiles, ragged tails in every dimension,
 # empty groups, groups shorter than one MMA step.
 SMALL = [
@@ -37,7 +46,7 @@ def _inputs(G, N, K, m, seed, bias=True, device="cuda"):
 
 @pytest.mark.parametrize("G,N,K,m", SMALL)
 @pytest.mark.parametrize("per_group", [False, True])
-def test_fwd_dgrad_wgrad_small(G, N, K, m, per_group):
+def test_fwd_dgrad_wgrad_small(G, N, K, m, per_group, tile_mode):
     M = int(sum(m))
     d = _inputs(G, N, K, m, seed=G * 7 + N)
     off, st = offsets_on_device(m, M, M + 64)
@@ -74,7 +83,7 @@ def test_fwd_dgrad_wgrad_small(G, N, K, m, per_group):
             assert orc.rel_frobenius(got_over[g], ref_over[g]) <= TOL_BF16, g
 
 
-def test_integer_mode_bit_exact():
+def test_integer_mode_bit_exact(tile_mode):
     """{-1,0,1} operands and integer biases: every sum is exact, so the GPU
     must reproduce the oracle bit for bit (tiny workload shapes)."""
     G, N, K, m = 4, 256, 128, [0, 96, 160, 256]
@@ -120,7 +129,7 @@ def test_caller_buffer_matches_internal_allocation():
     assert untouched(y_buf[M:])
 
 
-def test_many_groups_per_group_chunking():
+def test_many_groups_per_group_chunking(tile_mode):
     """More groups than one launch carries in per-group mode (64)."""
     rng = np.random.default_rng(9)
     G, N, K = 150, 136, 64
@@ -143,7 +152,7 @@ def test_many_groups_per_group_chunking():
             assert orc.rel_frobenius(got[g] - mg0[g], ref[g] - mg0[g]) <= TOL_BF16
 
 
-def test_all_groups_empty():
+def test_all_groups_empty(tile_mode):
     G, N, K, m = 3, 256, 128, [0, 0, 0]
     d = synth.operands(G, 8, N, K, 1)
     x = d["x"].cuda()[:0]      # zero rows, but a valid base pointer
@@ -246,6 +255,6 @@ def _sampled_parity(name):
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled(name):
+def test_full_size_sampled(name, tile_mode):
     _sampled_parity(name)
     torch.cuda.empty_cache()
