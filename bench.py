@@ -225,8 +225,8 @@ def dist_setup(gpus: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=[w for w in synth.WORKLOADS if w != "mxfp8_g8"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -269,16 +269,11 @@ def main():
     step = Step(args.workload, seed_offset=rank, device=dev)
     pk = peaks()
 
-    for _ in range(max(args.warmup, 3)):
-        step.run()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
+    sampler.start()  # sample clocks through warm-up and the timed region
+    for _ in range(max(args.warmup, 3)):
+        step.run()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()

@@ -41,6 +41,7 @@ constexpr int BK = 64;  // contraction elements per stage (one 128-byte swizzle 
 constexpr int kThreads = 192;
 constexpr int kPG = 64;  // per-group tensor maps carried by one launch
 constexpr int kSmemBudget = 196608;
+constexpr int kBand = 8;  // tile rows per rasterisation band
 
 template <int MODE, int CG>
 struct Cfg {
@@ -124,17 +125,22 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const Gemm
   const int local = t - prefix[lo];
   const int64_t o0 = __ldg(p.offsets + lo), o1 = __ldg(p.offsets + lo + 1);
   const int64_t m = o1 > o0 ? o1 - o0 : 0;
+  // Tile grid of the group: mtg x ntg.  Rasterise in bands of kBand tile
+  // rows, column-major inside a band, so the ~#SMs tiles in flight cover a
+  // near-square block and share operand strips through L2.
+  const int mtg = (MODE == kWgrad) ? ceil_div_i(p.N, C::kTileM) : ceil_div_i(m, C::kTileM);
+  const int ntg = ceil_div_i(MODE == kFwd ? p.N : p.K, C::kTileN);
+  const int band = local / (kBand * ntg);
+  const int base_mt = band * kBand;
+  const int bh = min(kBand, mtg - base_mt);
+  const int within = local - band * kBand * ntg;
+  tl.mt = base_mt + within % bh;
+  tl.nt = within / bh;
   if (MODE == kWgrad) {
-    const int mtn = ceil_div_i(p.N, C::kTileM);
-    tl.mt = local % mtn;
-    tl.nt = local / mtn;
     tl.r0 = o0;
     tl.r1 = o0 + m;
     tl.num_kb = ceil_div_i(m, BK);
   } else {
-    const int mtg = ceil_div_i(m, C::kTileM);
-    tl.mt = local % mtg;  // m-tiles fastest: neighbouring CTAs share a weight strip
-    tl.nt = local / mtg;
     tl.r0 = o0 + static_cast<int64_t>(tl.mt) * C::kTileM;
     tl.r1 = o0 + m;
     tl.num_kb = ceil_div_i(MODE == kFwd ? p.K : p.N, BK);
