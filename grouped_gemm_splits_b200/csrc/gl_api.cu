@@ -163,22 +163,139 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
   return gl::launch_grouped_gemm(c);
 }
 
+// ---------------------------------------------------------------- MXFP8 GEMMs
+static gl_status check_mx_dims(int G, int64_t M, int N, int K) {
+  if (G <= 0 || G > GL_MAX_GROUPS_MXFP8 || M < 0 || N <= 0 || K <= 0) return GL_ERR_INVALID;
+  if (N % 128 != 0 || K % 128 != 0) return GL_ERR_UNSUPPORTED;
+  if (M >= (int64_t(1) << 31)) return GL_ERR_UNSUPPORTED;
+  const int64_t rt = (M + 127) / 128 + G;
+  const int64_t ct = (int64_t(N > K ? N : K) + 127) / 128;
+  if (rt * ct >= (int64_t(1) << 31) || int64_t(G) * ct * ct >= (int64_t(1) << 31)) return GL_ERR_UNSUPPORTED;
+  return GL_OK;
+}
+
+gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_grouped w_codes,
+                       gl_grouped w_scales, const gl_grouped* bias, const int64_t* offsets,
+                       int32_t* status, int G, int64_t M, int N, int K, void* y, int64_t y_rows,
+                       void* stream) {
+  gl_status st = check_mx_dims(G, M, N, K);
+  if (st != GL_OK) return st;
+  if (((x_codes == nullptr || x_scales == nullptr || y == nullptr) && M > 0) || offsets == nullptr ||
+      status == nullptr)
+    return GL_ERR_INVALID;
+  if (!grouped_ok(w_codes, G) || !grouped_ok(w_scales, G) || (bias && !grouped_ok(*bias, G)))
+    return GL_ERR_INVALID;
+  if (y_rows < M) return GL_ERR_INVALID;
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(y) || !grouped_aligned(w_codes, G) ||
+      !grouped_aligned(w_scales, G) || (bias && !grouped_aligned(*bias, G)))
+    return GL_ERR_UNSUPPORTED;
+  if (M == 0) return GL_OK;
+  gl::MxCall c{};
+  c.mode = gl::kFwd;
+  c.a = x_codes;
+  c.sa = x_scales;
+  c.w = w_codes;
+  c.ws = w_scales;
+  c.bias = bias;
+  c.out = y;
+  c.out_rows = y_rows;
+  c.offsets = offsets;
+  c.status = status;
+  c.G = G;
+  c.M = M;
+  c.N = N;
+  c.K = K;
+  c.stream = to_stream(stream);
+  return gl::launch_grouped_gemm_mx(c);
+}
+
+gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_grouped w_codes_c,
+                         gl_grouped w_scales_c, const int64_t* offsets, int32_t* status, int G,
+                         int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream) {
+  gl_status st = check_mx_dims(G, M, N, K);
+  if (st != GL_OK) return st;
+  if (((dy_codes == nullptr || dy_scales == nullptr || dx == nullptr) && M > 0) || offsets == nullptr ||
+      status == nullptr)
+    return GL_ERR_INVALID;
+  if (!grouped_ok(w_codes_c, G) || !grouped_ok(w_scales_c, G)) return GL_ERR_INVALID;
+  if (dx_rows < M) return GL_ERR_INVALID;
+  if (!aligned16(dy_codes) || !aligned16(dy_scales) || !aligned16(dx) || !grouped_aligned(w_codes_c, G) ||
+      !grouped_aligned(w_scales_c, G))
+    return GL_ERR_UNSUPPORTED;
+  if (M == 0) return GL_OK;
+  gl::MxCall c{};
+  c.mode = gl::kDgrad;
+  c.a = dy_codes;
+  c.sa = dy_scales;
+  c.w = w_codes_c;
+  c.ws = w_scales_c;
+  c.out = dx;
+  c.out_rows = dx_rows;
+  c.offsets = offsets;
+  c.status = status;
+  c.G = G;
+  c.M = M;
+  c.N = N;
+  c.K = K;
+  c.stream = to_stream(stream);
+  return gl::launch_grouped_gemm_mx(c);
+}
+
+gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, const uint8_t* dy_codes_c,
+                         const uint8_t* dy_scales_c, const int64_t* offsets, int32_t* status, int G,
+                         int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream) {
+  gl_status st = check_mx_dims(G, M, N, K);
+  if (st != GL_OK) return st;
+  if (((x_codes_c == nullptr || x_scales_c == nullptr || dy_codes_c == nullptr || dy_scales_c == nullptr) &&
+       M > 0) ||
+      offsets == nullptr || status == nullptr)
+    return GL_ERR_INVALID;
+  if (!grouped_ok(main_grad, G)) return GL_ERR_INVALID;
+  if (!aligned16(x_codes_c) || !aligned16(x_scales_c) || !aligned16(dy_codes_c) || !aligned16(dy_scales_c) ||
+      !grouped_aligned(main_grad, G))
+    return GL_ERR_UNSUPPORTED;
+  if (M == 0) {
+    if (accumulate) return GL_OK;
+    const void* any = main_grad.mode == GL_STACKED ? main_grad.base : main_grad.ptrs[0];
+    x_codes_c = x_scales_c = dy_codes_c = dy_scales_c = static_cast<const uint8_t*>(any);
+  }
+  gl::MxCall c{};
+  c.mode = gl::kWgrad;
+  c.a = dy_codes_c;
+  c.sa = dy_scales_c;
+  c.b = x_codes_c;
+  c.sb = x_scales_c;
+  c.out_grouped = main_grad;
+  c.offsets = offsets;
+  c.status = status;
+  c.G = G;
+  c.M = M;
+  c.N = N;
+  c.K = K;
+  c.accumulate = accumulate ? 1 : 0;
+  c.stream = to_stream(stream);
+  return gl::launch_grouped_gemm_mx(c);
+}
+
 gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                                int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
-                               uint8_t* codes_c, uint8_t* scales_c, void* stream) {
+                               uint8_t* codes_c, uint8_t* scales_c, int scale_layout, void* stream) {
   if (src == nullptr || rows < 0 || cols <= 0 || G <= 0 || G > GL_MAX_GROUPS) return GL_ERR_INVALID;
   if (codes_r == nullptr && codes_c == nullptr) return GL_ERR_INVALID;
   if ((codes_r != nullptr) != (scales_r != nullptr) && codes_r != nullptr) return GL_ERR_INVALID;
   if (codes_r != nullptr && scales_r == nullptr) return GL_ERR_INVALID;
   if (codes_c != nullptr && scales_c == nullptr) return GL_ERR_INVALID;
   if (cols % 32 != 0) return GL_ERR_UNSUPPORTED;
+  if (scale_layout != GL_SCALES_ROWMAJOR && scale_layout != GL_SCALES_KGROUP) return GL_ERR_INVALID;
+  if (scale_layout == GL_SCALES_KGROUP && cols % 128 != 0) return GL_ERR_UNSUPPORTED;
+  if (rows >= (int64_t(1) << 31)) return GL_ERR_UNSUPPORTED;
   if (row_offsets == nullptr && rows % G != 0) return GL_ERR_INVALID;
   if (!aligned16(src) || (codes_r && (reinterpret_cast<uintptr_t>(codes_r) & 7u)) ||
       (codes_c && (reinterpret_cast<uintptr_t>(codes_c) & 7u)))
     return GL_ERR_UNSUPPORTED;
   if (rows == 0) return GL_OK;
   return gl::launch_quantize(src, rows, cols, row_offsets, G, status, codes_r, scales_r, codes_c,
-                             scales_c, to_stream(stream));
+                             scales_c, scale_layout, to_stream(stream));
 }
 
 }  // extern "C"

@@ -45,11 +45,35 @@ struct GemmCall {
 
 gl_status launch_grouped_gemm(const GemmCall& c);
 
+// MXFP8 grouped GEMM (E4M3 codes, E8M0 scales; see gl_gemm_mx.cu).
+struct MxCall {
+  int mode;
+  const void* a;           // A codes: FWD x, DGRAD dy (rowwise); WGRAD dy (columnwise)
+  const void* sa;          // A scales: k-group rowwise (FWD/DGRAD) or columnwise [S, N] (WGRAD)
+  const void* b;           // WGRAD: x columnwise codes
+  const void* sb;          // WGRAD: x columnwise scales [S, K]
+  gl_grouped w;            // FWD: W rowwise codes; DGRAD: W columnwise codes
+  gl_grouped ws;           // FWD: W k-group rowwise scales; DGRAD: W columnwise scales
+  const gl_grouped* bias;  // FWD (nullable)
+  gl_grouped out_grouped;  // WGRAD main_grad
+  void* out;
+  int64_t out_rows;
+  const int64_t* offsets;
+  int32_t* status;
+  int G;
+  int64_t M;
+  int N, K;
+  int accumulate;
+  cudaStream_t stream;
+};
+
+gl_status launch_grouped_gemm_mx(const MxCall& c);
+
 gl_status launch_offsets(const int64_t* m, int G, int64_t expect_rows, int64_t out_rows,
                          int64_t* offsets, int32_t* status, cudaStream_t stream);
 
 gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                           int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
-                          uint8_t* codes_c, uint8_t* scales_c, cudaStream_t stream);
+                          uint8_t* codes_c, uint8_t* scales_c, int scale_layout, cudaStream_t stream);
 
 }  // namespace gl

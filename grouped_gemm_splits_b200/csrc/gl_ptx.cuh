@@ -336,3 +336,51 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_ma
 }
 
 }  // namespace gl
+
+namespace gl {
+
+// ---------------------------------------------------------------- block-scaled MMA
+// D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T with E4M3 A/B in shared memory and
+// E8M0 scale factors in TMEM (kind::mxf8f6f4, one scale per 32 K-elements).
+__device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy 32 rows x 16 bytes of shared memory into TMEM (lanes 0-31, replicated
+// to all four lane quarters), 4 columns starting at taddr.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Descriptor of a contiguous 512-byte [32 rows x 16 bytes] shared-memory block
+// (no swizzle; 8-row core matrices 128 bytes apart) for tcgen05.cp.
+__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(512u >> 4) << 16;  // leading offset (unused: one 16-byte column)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;  // stride between 8-row core matrices
+  d |= 1ull << 46;                               // descriptor version for sm_100
+  return d;                                      // layout type 0: no swizzle
+}
+
+// Instruction descriptor, kind::mxf8f6f4 block-scaled, E4M3 A/B, E8M0 scales.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, int a_mn, int b_mn, int a_sf, int b_sf) {
+  return (static_cast<uint32_t>(b_sf & 3) << 4)     // B scale-factor byte
+         | (0u << 7) | (0u << 10)                   // A, B format: E4M3
+         | (static_cast<uint32_t>(a_mn) << 15)      // A major
+         | (static_cast<uint32_t>(b_mn) << 16)      // B major
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (1u << 23)                               // scale format: E8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)    // M / 16
+         | (static_cast<uint32_t>(a_sf & 3) << 29); // A scale-factor byte
+}
+
+}  // namespace gl

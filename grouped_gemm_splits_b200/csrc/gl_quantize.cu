@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kQThreads)
     quantize_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int cols,
                     const int64_t* __restrict__ row_offsets, int G, const int32_t* __restrict__ status,
                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r,
-                    uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c) {
+                    uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, int kgroup_pitch) {
   extern __shared__ int64_t qsmem[];
   int64_t* bprefix = qsmem;  // G+1: first block index of each group (ragged mode)
   __shared__ float cmax[kQThreads / 32][kQCols];
@@ -157,7 +157,15 @@ __global__ void __launch_bounds__(kQThreads)
           q.x = e4m3x4(v[i][0] * s, v[i][1] * s, v[i][2] * s, v[i][3] * s);
           q.y = e4m3x4(v[i][4] * s, v[i][5] * s, v[i][6] * s, v[i][7] * s);
           *reinterpret_cast<uint2*>(codes_r + row * cols + col) = q;
-          if ((c8 & 3) == 0) scales_r[row * (cols / 32) + col / 32] = static_cast<uint8_t>(e + 127);
+          if ((c8 & 3) == 0) {
+            // row-major [rows, cols/32], or k-group-major words: the four
+            // scales of k-blocks 4j..4j+3 of a row form word (j, row) of a
+            // [cols/128][kgroup_pitch] array (what the MXFP8 GEMM loads per stage)
+            const int64_t kb = col / 32;
+            const int64_t at = kgroup_pitch > 0 ? ((kb >> 2) * kgroup_pitch + row) * 4 + (kb & 3)
+                                                : row * (cols / 32) + kb;
+            scales_r[at] = static_cast<uint8_t>(e + 127);
+          }
         }
       }
     }
@@ -206,14 +214,14 @@ __global__ void __launch_bounds__(kQThreads)
 
 gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                           int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
-                          uint8_t* codes_c, uint8_t* scales_c, cudaStream_t stream) {
+                          uint8_t* codes_c, uint8_t* scales_c, int scale_layout, cudaStream_t stream) {
   const int smem = row_offsets != nullptr ? (G + 1) * static_cast<int>(sizeof(int64_t)) : 0;
   if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel), smem + 16 * 1024) != cudaSuccess)
     return GL_ERR_CUDA;
   const int grid = num_sms() * 8;
   quantize_kernel<<<grid, kQThreads, smem, stream>>>(
       static_cast<const __nv_bfloat16*>(src), rows, cols, row_offsets, G, status, codes_r,
-      scales_r, codes_c, scales_c);
+      scales_r, codes_c, scales_c, scale_layout == GL_SCALES_KGROUP ? static_cast<int>((rows + 3) / 4 * 4) : 0);
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
 }
 

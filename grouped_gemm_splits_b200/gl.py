@@ -21,9 +21,10 @@ _lib = None
 GL_OK, GL_ERR_INVALID, GL_ERR_UNSUPPORTED, GL_ERR_CUDA = 0, 1, 2, 3
 GL_DEV_NEG_SPLIT, GL_DEV_SUM_MISMATCH, GL_DEV_OUT_OVERFLOW, GL_DEV_TIMEOUT = 1, 2, 4, 8
 GL_STACKED, GL_PER_GROUP = 0, 1
+GL_SCALES_ROWMAJOR, GL_SCALES_KGROUP = 0, 1
 
 EXPORTED = ("gl_version", "gl_status_string", "gl_set_cta_pair", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
-            "group_quantize_mxfp8")
+            "group_quantize_mxfp8", "gl_fwd_mxfp8", "gl_dgrad_mxfp8", "gl_wgrad_mxfp8")
 
 
 class GlGrouped(ctypes.Structure):
@@ -62,7 +63,14 @@ def load() -> ctypes.CDLL:
     L.gl_wgrad.restype = i32
     L.gl_wgrad.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, vp]
     L.group_quantize_mxfp8.restype = i32
-    L.group_quantize_mxfp8.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, vp, vp, vp]
+    L.group_quantize_mxfp8.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, vp, vp, i32, vp]
+    L.gl_fwd_mxfp8.restype = i32
+    L.gl_fwd_mxfp8.argtypes = [vp, vp, GlGrouped, GlGrouped, ctypes.POINTER(GlGrouped), vp, vp, i32, i64, i32,
+                               i32, vp, i64, vp]
+    L.gl_dgrad_mxfp8.restype = i32
+    L.gl_dgrad_mxfp8.argtypes = [vp, vp, GlGrouped, GlGrouped, vp, vp, i32, i64, i32, i32, vp, i64, vp]
+    L.gl_wgrad_mxfp8.restype = i32
+    L.gl_wgrad_mxfp8.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, vp]
     _lib = L
     return L
 
@@ -176,13 +184,21 @@ def colwise_scale_rows_bound(rows: int, G: int) -> int:
     return (rows + 31) // 32 + G
 
 
+def kgroup_pitch(rows: int) -> int:
+    """Row pitch (in 4-byte words) of k-group-major rowwise scales."""
+    return (rows + 3) // 4 * 4
+
+
 def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] = None, G: int = 1,
                          rowwise: bool = True, colwise: bool = False,
-                         status: Optional[torch.Tensor] = None, out: Optional[dict] = None) -> dict:
+                         status: Optional[torch.Tensor] = None, out: Optional[dict] = None,
+                         kgroup_scales: bool = False) -> dict:
     """MXFP8 cast of a bf16 [rows, cols] tensor (rows in G groups).
 
     Returns a dict with ``codes_r``/``scales_r`` (blocks along each row) and/or
-    ``codes_c``/``scales_c`` (blocks of 32 rows inside each group).
+    ``codes_c``/``scales_c`` (blocks of 32 rows inside each group).  With
+    ``kgroup_scales`` the rowwise scales are a [cols/128, pitch, 4] array (the
+    form the MXFP8 GEMMs read) instead of [rows, cols/32].
     """
     if src.dim() == 3:
         G = src.shape[0]
@@ -196,7 +212,11 @@ def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] 
     out = {} if out is None else out
     if rowwise:
         out.setdefault("codes_r", torch.empty(rows, cols, dtype=torch.uint8, device=dev))
-        out.setdefault("scales_r", torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev))
+        if kgroup_scales:
+            out.setdefault("scales_r", torch.empty(cols // 128, kgroup_pitch(rows), 4, dtype=torch.uint8,
+                                                   device=dev))
+        else:
+            out.setdefault("scales_r", torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev))
     if colwise:
         out.setdefault("codes_c", torch.empty(rows, cols, dtype=torch.uint8, device=dev))
         out.setdefault("scales_c", torch.empty(colwise_scale_rows_bound(rows, G), cols,
@@ -205,5 +225,74 @@ def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] 
         src2.data_ptr(), rows, cols, _ptr(row_offsets), G, _ptr(status),
         _ptr(out.get("codes_r")) if rowwise else None, _ptr(out.get("scales_r")) if rowwise else None,
         _ptr(out.get("codes_c")) if colwise else None, _ptr(out.get("scales_c")) if colwise else None,
-        _stream()), "group_quantize_mxfp8")
+        GL_SCALES_KGROUP if kgroup_scales else GL_SCALES_ROWMAJOR, _stream()), "group_quantize_mxfp8")
     return out
+
+
+# ---------------------------------------------------------------- MXFP8 GEMMs
+
+def _grouped_any(t: TensorOrList, G: int):
+    """gl_grouped for a stacked tensor (any leading shape) or a list of G tensors."""
+    if isinstance(t, torch.Tensor):
+        assert t.is_contiguous()
+        return GlGrouped(GL_STACKED, t.data_ptr(), None), None
+    assert len(t) == G
+    arr = (ctypes.c_void_p * G)(*[x.data_ptr() for x in t])
+    return GlGrouped(GL_PER_GROUP, None, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))), arr
+
+
+def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorOrList, w_scales: TensorOrList,
+                 bias: Optional[TensorOrList], offsets: torch.Tensor, status: torch.Tensor,
+                 y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """fprop on MXFP8 operands: x rowwise codes [M,K] + k-group scales; W rowwise
+    codes [G,N,K] (or G x [N,K]) + k-group scales."""
+    G = offsets.numel() - 1
+    M, K = x_codes.shape
+    N = (w_codes if isinstance(w_codes, torch.Tensor) else w_codes[0]).shape[-2]
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x_codes.device)
+    wc, k1 = _grouped_any(w_codes, G)
+    ws, k2 = _grouped_any(w_scales, G)
+    bptr, k3 = None, None
+    if bias is not None:
+        bg, k3 = _grouped(bias, G)
+        bptr = ctypes.pointer(bg)
+    _check(load().gl_fwd_mxfp8(x_codes.data_ptr(), x_scales.data_ptr(), wc, ws, bptr, offsets.data_ptr(),
+                               status.data_ptr(), G, M, N, K, y.data_ptr(), y.shape[0], _stream()),
+           "gl_fwd_mxfp8")
+    del k1, k2, k3
+    return y
+
+
+def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: TensorOrList,
+                   w_scales_c: TensorOrList, offsets: torch.Tensor, status: torch.Tensor,
+                   dx: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """dgrad on MXFP8 operands: dy rowwise codes [M,N] + k-group scales; W
+    columnwise codes [G,N,K] + columnwise scales."""
+    G = offsets.numel() - 1
+    M, N = dy_codes.shape
+    K = (w_codes_c if isinstance(w_codes_c, torch.Tensor) else w_codes_c[0]).shape[-1]
+    if dx is None:
+        dx = torch.empty(M, K, dtype=torch.bfloat16, device=dy_codes.device)
+    wc, k1 = _grouped_any(w_codes_c, G)
+    ws, k2 = _grouped_any(w_scales_c, G)
+    _check(load().gl_dgrad_mxfp8(dy_codes.data_ptr(), dy_scales.data_ptr(), wc, ws, offsets.data_ptr(),
+                                 status.data_ptr(), G, M, N, K, dx.data_ptr(), dx.shape[0], _stream()),
+           "gl_dgrad_mxfp8")
+    del k1, k2
+    return dx
+
+
+def gl_wgrad_mxfp8(x_codes_c: torch.Tensor, x_scales_c: torch.Tensor, dy_codes_c: torch.Tensor,
+                   dy_scales_c: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
+                   main_grad: TensorOrList, accumulate: bool = True) -> TensorOrList:
+    """wgrad on MXFP8 operands: x and dy columnwise codes + columnwise scales."""
+    G = offsets.numel() - 1
+    M, K = x_codes_c.shape
+    N = dy_codes_c.shape[1]
+    mg, keep = _grouped(main_grad, G)
+    _check(load().gl_wgrad_mxfp8(x_codes_c.data_ptr(), x_scales_c.data_ptr(), dy_codes_c.data_ptr(),
+                                 dy_scales_c.data_ptr(), offsets.data_ptr(), status.data_ptr(), G, M, N, K, mg,
+                                 1 if accumulate else 0, _stream()), "gl_wgrad_mxfp8")
+    del keep
+    return main_grad

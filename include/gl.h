@@ -185,7 +185,12 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
  *   status      device int32 status word or NULL; non-zero -> nothing written
  *   codes_r     NULL or device u8 [rows, cols]: rowwise codes (blocks of 32
  *               along each row)
- *   scales_r    device u8 [rows, cols/32] (required with codes_r)
+ *   scales_r    device u8 (required with codes_r): with scale_layout ==
+ *               GL_SCALES_ROWMAJOR a [rows, cols/32] array; with
+ *               GL_SCALES_KGROUP (cols % 128 == 0) a [cols/128][P][4] array,
+ *               P = rows rounded up to a multiple of 4, whose element
+ *               (j, r, b) is the scale of k-block 4j+b of row r -- the form
+ *               the MXFP8 GEMMs read (one contiguous box per stage)
  *   codes_c     NULL or device u8 [rows, cols]: columnwise codes (blocks of 32
  *               rows along each column, restarting at every group's first
  *               row; a group's last block may be partial)
@@ -194,9 +199,49 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
  *               S <= ceil(rows/32) + G bounds the rows used.
  * Limits: cols % 32 == 0; rows/G integral when row_offsets is NULL.
  */
+#define GL_SCALES_ROWMAJOR 0
+#define GL_SCALES_KGROUP 1
 gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                                int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
-                               uint8_t* codes_c, uint8_t* scales_c, void* stream);
+                               uint8_t* codes_c, uint8_t* scales_c, int scale_layout, void* stream);
+
+/*
+ * MXFP8 grouped GEMMs -- the three products of gl_fwd / gl_dgrad / gl_wgrad
+ * on MXFP8 operands (E4M3 codes, E8M0 scale per 32 contraction elements, as
+ * written by group_quantize_mxfp8), computed as
+ *     sum over k of (q_a * 2^(s_a - 127)) * (q_b * 2^(s_b - 127))
+ * with fp32 accumulation on the block-scaled tensor cores (``grouped_linear.py``
+ * fuser_forward / fuser_backward with MXFP8 quantizers: x and W rowwise for
+ * fprop, dy rowwise and W columnwise for dgrad, x and dy columnwise for wgrad).
+ * Outputs, offsets, status, caller buffers and main_grad behave exactly as in
+ * the bf16 entry points.
+ *
+ * Operand forms (all device memory, produced by group_quantize_mxfp8):
+ *   rowwise codes    u8 [rows, cols] (x, dy: [M, K] / [M, N]; W: [G, N, K])
+ *   k-group scales   GL_SCALES_KGROUP rowwise scales, [cols/128][P][4] with
+ *                    P = rows rounded up to 4 (x: cols K, rows M; dy: cols N,
+ *                    rows M; stacked W: cols K, rows G*N; per-group W: rows N)
+ *   columnwise codes u8 [rows, cols] (x_c [M, K], dy_c [M, N], W_c [G, N, K])
+ *   columnwise scales u8 [S, cols] as group_quantize_mxfp8 writes them: for
+ *                    x_c / dy_c quantized with the group offsets, S >=
+ *                    ceil(M/32) + G rows allocated; for W_c (equal groups of
+ *                    N rows) G * ceil(N/32) rows, or ceil(N/32) per group.
+ * Limits: N % 128 == 0, K % 128 == 0, G <= GL_MAX_GROUPS_MXFP8.
+ */
+#define GL_MAX_GROUPS_MXFP8 2048
+
+gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_grouped w_codes,
+                       gl_grouped w_scales, const gl_grouped* bias, const int64_t* offsets,
+                       int32_t* status, int G, int64_t M, int N, int K, void* y, int64_t y_rows,
+                       void* stream);
+
+gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_grouped w_codes_c,
+                         gl_grouped w_scales_c, const int64_t* offsets, int32_t* status, int G,
+                         int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream);
+
+gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, const uint8_t* dy_codes_c,
+                         const uint8_t* dy_scales_c, const int64_t* offsets, int32_t* status, int G,
+                         int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream);
 
 #ifdef __cplusplus
 }

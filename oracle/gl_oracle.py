@@ -297,6 +297,19 @@ def quantize_rowwise(src: np.ndarray):
     return codes.reshape(rows, cols), (e + 127).astype(np.uint8)
 
 
+def rowwise_scales_kgroup(scales: np.ndarray) -> np.ndarray:
+    """Rowwise scales [rows, cols/32] rearranged k-group-major: element
+    (j, r, b) = scales[r, 4j + b], shape [cols/128, rows, 4] (the library pads
+    the row dimension to a multiple of 4; padding is not compared)."""
+    rows, nb = scales.shape
+    assert nb % 4 == 0
+    out = np.zeros((nb // 4, rows, 4), dtype=np.uint8)
+    for j in range(nb // 4):
+        for b in range(4):
+            out[j, :, b] = scales[:, 4 * j + b]
+    return out
+
+
 def colwise_scale_rows(m_splits) -> np.ndarray:
     """First scale row of each group in the columnwise scale array.
 

@@ -55,9 +55,12 @@ def test_host_side_validation_without_gpu():
     pg = gl.GlGrouped(gl.GL_PER_GROUP, None, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
     assert lib.gl_fwd(16, pg, None, 16, 16, 2, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
     # quantize: cols not a multiple of 32; no output requested
-    assert lib.group_quantize_mxfp8(16, 8, 48, None, 1, None, 16, 16, None, None, None) == gl.GL_ERR_UNSUPPORTED
-    assert lib.group_quantize_mxfp8(16, 8, 64, None, 1, None, None, None, None, None, None) == gl.GL_ERR_INVALID
-    assert lib.group_quantize_mxfp8(16, 9, 64, None, 2, None, 16, 16, None, None, None) == gl.GL_ERR_INVALID
+    assert lib.group_quantize_mxfp8(16, 8, 48, None, 1, None, 16, 16, None, None, 0, None) == gl.GL_ERR_UNSUPPORTED
+    assert lib.group_quantize_mxfp8(16, 8, 64, None, 1, None, None, None, None, None, 0, None) == gl.GL_ERR_INVALID
+    assert lib.group_quantize_mxfp8(16, 9, 64, None, 2, None, 16, 16, None, None, 0, None) == gl.GL_ERR_INVALID
+    # k-group-major scales need cols % 128 == 0; unknown layout codes are rejected
+    assert lib.group_quantize_mxfp8(16, 8, 96, None, 1, None, 16, 16, None, None, 1, None) == gl.GL_ERR_UNSUPPORTED
+    assert lib.group_quantize_mxfp8(16, 8, 128, None, 1, None, 16, 16, None, None, 7, None) == gl.GL_ERR_INVALID
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

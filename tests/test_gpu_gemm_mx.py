@@ -1,0 +1,183 @@
+"""MXFP8 grouped GEMMs on the GPU (through the C ABI) against the fp64 oracle.
+
+Both sides quantize the same bf16 inputs: the GPU with group_quantize_mxfp8
+(checked bit-exact against the oracle quantizer in test_gpu_quantize.py), the
+oracle with its own quantizer; the oracle then multiplies the dequantized
+operands in fp64.  Bar: relative Frobenius error <= 1e-2 per group; bit-exact
+in an integer-valued mode; caller-buffer tails untouched; accumulate and
+overwrite of main_grad as for bf16 (``grouped_linear.py`` fuser_forward /
+fuser_backward with MXFP8 quantizers).
+"""
+import numpy as np
+import pytest
+import torch
+
+from grouped_gemm_splits_b200 import gl, synth
+from oracle import gl_oracle as orc
+from tests.gpu_util import f64, offsets_on_device, sample_rows, sentinel_like, untouched
+
+pytestmark = pytest.mark.gpu
+
+TOL_MX = 1e-2
+
+
+def _quantize_all(d, m, G, N, K, off, st):
+    """GPU MXFP8 copies of x, W and dy in the forms the GEMMs read."""
+    q = {}
+    q["x"] = gl.group_quantize_mxfp8(d["x"], off, rowwise=True, colwise=True, status=st, kgroup_scales=True)
+    q["dy"] = gl.group_quantize_mxfp8(d["dy"], off, rowwise=True, colwise=True, status=st, kgroup_scales=True)
+    q["w"] = gl.group_quantize_mxfp8(d["w"], rowwise=True, colwise=True, kgroup_scales=True)  # G equal groups
+    return q
+
+
+def _oracle_all(d, m, G, N, K):
+    x, w, dy = f64(d["x"]), f64(d["w"]), f64(d["dy"])
+    xq, xs = orc.quantize_rowwise(x)
+    xcq, xcs = orc.quantize_colwise(x, m)
+    dyq, dys = orc.quantize_rowwise(dy)
+    dycq, dycs = orc.quantize_colwise(dy, m)
+    wq, ws = orc.quantize_rowwise(w.reshape(G * N, K))
+    wcq, wcs = orc.quantize_colwise(w.reshape(G * N, K), [N] * G)
+    return {
+        "fwd": orc.fwd_mxfp8(xq, xs, wq.reshape(G, N, K), ws.reshape(G, N, K // 32),
+                             f64(d["bias"]) if "bias" in d else None, m),
+        "dgrad": orc.dgrad_mxfp8(dyq, dys, wcq.reshape(G, N, K), wcs, m),
+        "wgrad_over": orc.wgrad_mxfp8(xcq, xcs, dycq, dycs, m, None, False),
+    }
+
+
+SMALL = [
+    (4, 256, 128, [0, 96, 160, 256]),
+    (5, 384, 512, [130, 0, 301, 7, 262]),
+    (1, 256, 256, [300]),
+    (8, 128, 256, [1, 15, 17, 63, 64, 65, 0, 130]),
+    (3, 512, 384, [257, 0, 511]),
+]
+
+
+@pytest.mark.parametrize("G,N,K,m", SMALL)
+@pytest.mark.parametrize("per_group", [False, True])
+def test_mxfp8_small(G, N, K, m, per_group):
+    M = int(sum(m))
+    d = {k: v.cuda() for k, v in synth.operands(G, M, N, K, seed=G + N + K, bias=True).items()}
+    off, st = offsets_on_device(m, M, M + 32)
+    q = _quantize_all(d, m, G, N, K, off, st)
+    if per_group:
+        wc = [q["w"]["codes_r"][g * N:(g + 1) * N].contiguous() for g in range(G)]
+        # per-group k-group scales: [K/128, pitch(N), 4] for each group
+        ws_full = q["w"]["scales_r"]
+        ws = [ws_full[:, g * N:(g + 1) * N].contiguous() for g in range(G)]
+        wcc = [q["w"]["codes_c"][g * N:(g + 1) * N].contiguous() for g in range(G)]
+        n32 = (N + 31) // 32
+        wcs = [q["w"]["scales_c"][g * n32:(g + 1) * n32].contiguous() for g in range(G)]
+        bias = [d["bias"][g].clone() for g in range(G)]
+    else:
+        wc = q["w"]["codes_r"].view(G, N, K)
+        ws = q["w"]["scales_r"]
+        wcc = q["w"]["codes_c"].view(G, N, K)
+        wcs = q["w"]["scales_c"]
+        bias = d["bias"]
+    y = sentinel_like(M + 32, N)
+    gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], wc, ws, bias, off, st, y)
+    dx = sentinel_like(M + 32, K)
+    gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], wcc, wcs, off, st, dx)
+    mg = torch.full((G, N, K), float("nan"), device="cuda")
+    mg_arg = [mg[g] for g in range(G)] if per_group else mg
+    gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
+                      mg_arg, accumulate=False)
+    mga = d["main_grad"].clone()
+    gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
+                      mga, accumulate=True)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = _oracle_all(d, m, G, N, K)
+    o = orc.offsets(m)
+    got_y, got_dx, got_w, got_a = f64(y), f64(dx), f64(mg), f64(mga)
+    mg0 = f64(d["main_grad"])
+    for g in range(G):
+        a, b = int(o[g]), int(o[g + 1])
+        if a == b:
+            assert np.all(got_w[g] == 0.0)
+            assert np.array_equal(got_a[g], mg0[g])
+            continue
+        assert orc.rel_frobenius(got_y[a:b], ref["fwd"][a:b]) <= TOL_MX, ("fwd", g)
+        assert orc.rel_frobenius(got_dx[a:b], ref["dgrad"][a:b]) <= TOL_MX, ("dgrad", g)
+        assert orc.rel_frobenius(got_w[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad", g)
+        assert orc.rel_frobenius(got_a[g] - mg0[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad acc", g)
+    assert untouched(y[M:]) and untouched(dx[M:])
+
+
+def test_mxfp8_integer_mode_bit_exact():
+    """Values in {-1,0,1}: every block scales by 2^-8 (or is all zero), the
+    codes are exact, and every product sum is an exact small integer."""
+    G, N, K, m = 3, 256, 128, [0, 100, 156]
+    M = sum(m)
+    d = {k: v.cuda() for k, v in synth.integer_operands(G, M, N, K, seed=3).items()}
+    off, st = offsets_on_device(m, M)
+    q = _quantize_all(d, m, G, N, K, off, st)
+    y = gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], q["w"]["codes_r"].view(G, N, K),
+                        q["w"]["scales_r"], d["bias"], off, st)
+    dx = gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], q["w"]["codes_c"].view(G, N, K),
+                           q["w"]["scales_c"], off, st)
+    mg = d["main_grad"].clone()
+    gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
+                      mg, accumulate=True)
+    torch.cuda.synchronize()
+    x64, w64, dy64 = f64(d["x"]), f64(d["w"]), f64(d["dy"])
+    assert np.array_equal(synth.bf16_bits(y), orc.f64_to_bf16_rne(orc.fwd(x64, w64, f64(d["bias"]), m)))
+    assert np.array_equal(f64(dx), orc.dgrad(dy64, w64, m))
+    assert np.array_equal(f64(mg), orc.wgrad(x64, dy64, m, f64(d["main_grad"]), True))
+
+
+def test_mxfp8_full_size_sampled():
+    """The MXFP8 workload (G=8, K=4096, N=14336, 16384 rows in multiples of
+    128) at full size; sampled entries against the oracle, which quantizes
+    exactly the rows / columns each entry needs."""
+    wl = synth.WORKLOADS["mxfp8_g8"]
+    m = synth.m_splits_for("mxfp8_g8")
+    G, N, K, M = wl.G, wl.N, wl.K, wl.rows
+    d = synth.operands(G, M, N, K, wl.seed, device="cuda", bias=False)
+    off, st = offsets_on_device(m, M)
+    q = _quantize_all(d, m, G, N, K, off, st)
+    y = gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], q["w"]["codes_r"].view(G, N, K),
+                        q["w"]["scales_r"], None, off, st)
+    dx = gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], q["w"]["codes_c"].view(G, N, K),
+                           q["w"]["scales_c"], off, st)
+    mg = torch.zeros(G, N, K, device="cuda")
+    gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
+                      mg, accumulate=False)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rng = np.random.default_rng(7)
+    o = orc.offsets(m)
+    rows = sample_rows(m, 2, rng)
+    grp = np.searchsorted(o, rows, side="right") - 1
+    got_f, ref_f, got_d, ref_d = [], [], [], []
+    for r, g in zip(rows, grp):
+        r, g = int(r), int(g)
+        xr = orc.dequant_rowwise(*orc.quantize_rowwise(f64(d["x"][r:r + 1])))[0]
+        dyr = orc.dequant_rowwise(*orc.quantize_rowwise(f64(d["dy"][r:r + 1])))[0]
+        for n in rng.integers(0, N, size=6):
+            wr = orc.dequant_rowwise(*orc.quantize_rowwise(f64(d["w"][g, int(n):int(n) + 1])))[0]
+            ref_f.append(orc.fwd_entry(xr, wr, None))
+            got_f.append(float(f64(y[r, int(n):int(n) + 1])[0]))
+        for k in rng.integers(0, K, size=6):
+            col = f64(d["w"][g][:, int(k):int(k) + 1])
+            wc = orc.dequant_colwise(*orc.quantize_colwise(col, [N]), [N])[:, 0]
+            ref_d.append(orc.dgrad_entry(dyr, wc))
+            got_d.append(float(f64(dx[r, int(k):int(k) + 1])[0]))
+    assert orc.rel_frobenius(np.array(got_f), np.array(ref_f)) <= TOL_MX
+    assert orc.rel_frobenius(np.array(got_d), np.array(ref_d)) <= TOL_MX
+    got_w, ref_w = [], []
+    for g in range(G):
+        a, b = int(o[g]), int(o[g + 1])
+        if a == b:
+            assert bool((mg[g] == 0).all())
+            continue
+        for _ in range(6):
+            n, k = int(rng.integers(N)), int(rng.integers(K))
+            dyc = orc.dequant_colwise(*orc.quantize_colwise(f64(d["dy"][a:b, n:n + 1]), [b - a]), [b - a])[:, 0]
+            xc = orc.dequant_colwise(*orc.quantize_colwise(f64(d["x"][a:b, k:k + 1]), [b - a]), [b - a])[:, 0]
+            ref_w.append(orc.wgrad_entry(dyc, xc, 0.0, False))
+            got_w.append(float(mg[g, n, k].item()))
+    assert orc.rel_frobenius(np.array(got_w), np.array(ref_w)) <= TOL_MX

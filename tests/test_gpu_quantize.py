@@ -41,6 +41,20 @@ def test_ragged_groups_bit_exact(m, cols):
     _check(src, m, got)
 
 
+@pytest.mark.parametrize("m,cols", [([0, 96, 160, 256], 128), ([5, 123, 0, 2], 384)])
+def test_kgroup_rowwise_scales(m, cols):
+    """The k-group-major rowwise scale layout holds the same bytes, permuted."""
+    rows = sum(m)
+    src = torch.randn(rows, cols, generator=torch.Generator().manual_seed(cols)).to(torch.bfloat16).cuda()
+    off, st = gl.gl_offsets(torch.tensor(m, dtype=torch.int64, device="cuda"), rows)
+    got = gl.group_quantize_mxfp8(src, off, rowwise=True, colwise=False, status=st, kgroup_scales=True)
+    torch.cuda.synchronize()
+    c, s = orc.quantize_rowwise(f64(src))
+    assert np.array_equal(got["codes_r"].cpu().numpy(), c)
+    assert got["scales_r"].shape == (cols // 128, gl.kgroup_pitch(rows), 4)
+    assert np.array_equal(got["scales_r"][:, :rows].cpu().numpy(), orc.rowwise_scales_kgroup(s))
+
+
 def test_every_bf16_value_bit_exact():
     """All 65536 bf16 patterns (finite ones), each alone in a 32-element block."""
     bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)

@@ -228,3 +228,12 @@ def test_planted_scale_mistake_is_caught():
         e_other = int(np.floor(np.log2(a))) - 8
         diffs += e_other + 127 != case["scale"]
     assert diffs > 0
+
+
+def test_kgroup_layout_is_a_permutation():
+    rng = np.random.default_rng(5)
+    sc = rng.integers(0, 256, (7, 12)).astype(np.uint8)
+    kg = orc.rowwise_scales_kgroup(sc)
+    assert kg.shape == (3, 7, 4)
+    assert sorted(kg.ravel().tolist()) == sorted(sc.ravel().tolist())
+    assert kg[2, 5, 1] == sc[5, 9] and kg[0, 0, 3] == sc[0, 3]
