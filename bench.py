@@ -106,8 +106,78 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # GPU step
 # ----------------------------------------------------------------------------
+class MxStep:
+    """The MXFP8 half of the step: cast x, W, dy (rowwise + columnwise), then
+    the three block-scaled GEMMs, on the MXFP8 workload (same shapes, splits
+    in multiples of 128)."""
+
+    NAMES = ["quant_x", "quant_w", "quant_dy", "fwd_mx", "dgrad_mx", "wgrad_mx"]
+
+    def __init__(self, seed_offset: int, device, x=None, w=None, dy=None, main_grad=None,
+                 workload: str = "mxfp8_g8"):
+        wl = synth.WORKLOADS[workload]
+        self.wl = wl
+        self.m = synth.m_splits_for(workload)
+        G, N, K, M = wl.G, wl.N, wl.K, wl.rows
+        if x is None:
+            d = synth.operands(G, M, N, K, wl.seed + seed_offset, device=device, bias=False)
+            x, w, dy, main_grad = d["x"], d["w"], d["dy"], d["main_grad"]
+        self.x, self.w, self.dy, self.main_grad = x, w, dy, main_grad
+        self.m_dev = torch.tensor(self.m, device=device)
+        self.offsets = torch.empty(G + 1, dtype=torch.int64, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        gl.gl_offsets(self.m_dev, M, M, self.offsets, self.status)
+        self.y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+        self.dx = torch.empty(M, K, dtype=torch.bfloat16, device=device)
+        self.qx, self.qw, self.qdy = {}, {}, {}
+        self.flops = 2.0 * float(self.m.sum()) * N * K
+        ne = int((self.m > 0).sum())
+        code_b = lambda n: n + n // 32  # codes + scales per copy
+        self.bytes = {
+            "quant_x": M * K * 2 + 2 * code_b(M * K),
+            "quant_w": G * N * K * 2 + 2 * code_b(G * N * K),
+            "quant_dy": M * N * 2 + 2 * code_b(M * N),
+            "fwd_mx": code_b(M * K) + code_b(ne * N * K) + M * N * 2,
+            "dgrad_mx": code_b(M * N) + code_b(ne * N * K) + M * K * 2,
+            "wgrad_mx": code_b(M * K) + code_b(M * N) + 2 * ne * N * K * 4,
+        }
+        self.launches = 6
+
+    def run(self, ev=None, i0=0):
+        wl = self.wl
+        G, N, K = wl.G, wl.N, wl.K
+        if ev:
+            ev[i0].record()
+        gl.gl_offsets(self.m_dev, wl.rows, wl.rows, self.offsets, self.status)
+        gl.group_quantize_mxfp8(self.x, self.offsets, rowwise=True, colwise=True, status=self.status,
+                                out=self.qx, kgroup_scales=True)
+        if ev:
+            ev[i0 + 1].record()
+        gl.group_quantize_mxfp8(self.w, rowwise=True, colwise=True, out=self.qw, kgroup_scales=True)
+        if ev:
+            ev[i0 + 2].record()
+        gl.group_quantize_mxfp8(self.dy, self.offsets, rowwise=True, colwise=True, status=self.status,
+                                out=self.qdy, kgroup_scales=True)
+        if ev:
+            ev[i0 + 3].record()
+        gl.gl_fwd_mxfp8(self.qx["codes_r"], self.qx["scales_r"], self.qw["codes_r"].view(G, N, K),
+                        self.qw["scales_r"], None, self.offsets, self.status, self.y)
+        if ev:
+            ev[i0 + 4].record()
+        gl.gl_dgrad_mxfp8(self.qdy["codes_r"], self.qdy["scales_r"], self.qw["codes_c"].view(G, N, K),
+                          self.qw["scales_c"], self.offsets, self.status, self.dx)
+        if ev:
+            ev[i0 + 5].record()
+        gl.gl_wgrad_mxfp8(self.qx["codes_c"], self.qx["scales_c"], self.qdy["codes_c"], self.qdy["scales_c"],
+                          self.offsets, self.status, self.main_grad, accumulate=True)
+        if ev:
+            ev[i0 + 6].record()
+
+
 class Step:
-    """Device buffers and one pass of the hot path on the current stream."""
+    """Device buffers and one pass of the whole hot path on the current stream:
+    offsets, bf16 fwd / dgrad / wgrad(accumulate), then the MXFP8 half
+    (cast of x, W, dy and the three block-scaled GEMMs)."""
 
     def __init__(self, workload: str, seed_offset: int, device):
         wl = synth.WORKLOADS[workload]
@@ -122,17 +192,27 @@ class Step:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.y = torch.empty(wl.out_rows, N, dtype=torch.bfloat16, device=device)
         self.dx = torch.empty(wl.out_rows, K, dtype=torch.bfloat16, device=device)
-        self.flops = 2.0 * float(self.m.sum()) * N * K  # per GEMM
-        # algorithmic bytes per launch (weights / main_grad of non-empty groups)
+        flops = 2.0 * float(self.m.sum()) * N * K  # per GEMM
         ne = int((self.m > 0).sum())
         xb, dyb = M * K * 2, M * N * 2
         wb, mgb = ne * N * K * 2, ne * N * K * 4
+        # the MXFP8 half: the MXFP8 workload's splits on the bf16 workload's
+        # tensors (same shapes), else this workload's own splits
+        mx_workload = "mxfp8_g8" if workload == "bf16_g8" else workload
+        self.mx = MxStep(seed_offset, device, self.x, self.w, self.dy, self.main_grad, workload=mx_workload)
+        self.names = ["offsets", "fwd", "dgrad", "wgrad"] + MxStep.NAMES
+        self.flops = {"fwd": flops, "dgrad": flops, "wgrad": flops,
+                      "fwd_mx": self.mx.flops, "dgrad_mx": self.mx.flops, "wgrad_mx": self.mx.flops}
         self.bytes = {"offsets": G * 8 + (G + 1) * 8 + 4,
                       "fwd": xb + wb + dyb, "dgrad": dyb + wb + xb, "wgrad": xb + dyb + 2 * mgb}
-        self.launches = 4
+        self.bytes.update(self.mx.bytes)
+        self.dtype = {"fwd": "bf16", "dgrad": "bf16", "wgrad": "bf16",
+                      "fwd_mx": "mxfp8", "dgrad_mx": "mxfp8", "wgrad_mx": "mxfp8"}
+        self.launches = 4 + self.mx.launches
+        self.total_flops = sum(self.flops.values())
 
     def run(self, ev=None):
-        """One step; ``ev`` = list of 5 events recorded around the four ops."""
+        """One step; ``ev`` = list of len(names)+1 events recorded around the ops."""
         if ev:
             ev[0].record()
         gl.gl_offsets(self.m_dev, self.wl.rows, self.wl.out_rows, self.offsets, self.status)
@@ -145,8 +225,7 @@ class Step:
         if ev:
             ev[3].record()
         gl.gl_wgrad(self.x, self.dy, self.offsets, self.status, self.main_grad, accumulate=True)
-        if ev:
-            ev[4].record()
+        self.mx.run(ev, 4)
 
 
 def e2e_measure(step: Step, steps: int, warmup: int):
@@ -159,10 +238,14 @@ def e2e_measure(step: Step, steps: int, warmup: int):
     h2d = hx.numel() * 2 + hdy.numel() * 2 + hm.numel() * 8
     d2h = 4
 
+    hm2 = torch.tensor(step.mx.m).pin_memory()
+    h2d += hm2.numel() * 8
+
     def one():
         step.x.copy_(hx, non_blocking=True)
         step.dy.copy_(hdy, non_blocking=True)
         step.m_dev.copy_(hm, non_blocking=True)
+        step.mx.m_dev.copy_(hm2, non_blocking=True)
         step.run()
         hst.copy_(step.status, non_blocking=True)
 
@@ -183,7 +266,7 @@ def e2e_measure(step: Step, steps: int, warmup: int):
 # ----------------------------------------------------------------------------
 # CPU oracle on a bounded sample
 # ----------------------------------------------------------------------------
-def oracle_sample(workload: str = WORKLOAD, seed_offset: int = 0, rows_per_group: int = 96, groups=(0, 1)):
+def oracle_sample(workload: str = WORKLOAD, seed_offset: int = 0, rows_per_group: int = 64, groups=(0, 1)):
     """fwd + dgrad + wgrad of the oracle on ``rows_per_group`` rows of two
     groups of the workload.  Returns (flops, seconds, threads, description)."""
     from oracle import gl_oracle as orc
@@ -201,11 +284,23 @@ def oracle_sample(workload: str = WORKLOAD, seed_offset: int = 0, rows_per_group
     orc.fwd(x, w, None, m)
     orc.dgrad(dy, w, m)
     orc.wgrad(x, dy, m, mg, True)
+    # the MXFP8 half: quantize (rowwise + columnwise), then the three products
+    Gs = len(gsel)
+    xq, xs = orc.quantize_rowwise(x)
+    xcq, xcs = orc.quantize_colwise(x, m)
+    dyq, dys = orc.quantize_rowwise(dy)
+    dycq, dycs = orc.quantize_colwise(dy, m)
+    wq, ws = orc.quantize_rowwise(w.reshape(Gs * N, K))
+    wcq, wcs = orc.quantize_colwise(w.reshape(Gs * N, K), [N] * Gs)
+    orc.fwd_mxfp8(xq, xs, wq.reshape(Gs, N, K), ws.reshape(Gs, N, K // 32), None, m)
+    orc.dgrad_mxfp8(dyq, dys, wcq.reshape(Gs, N, K), wcs, m)
+    orc.wgrad_mxfp8(xcq, xcs, dycq, dycs, m, mg, True)
     sec = time.perf_counter() - t0
-    flops = 3 * 2.0 * M * N * K
+    flops = 6 * 2.0 * M * N * K
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     desc = (f"{len(gsel)} groups x {rows_per_group} rows of the {workload} workload "
-            f"(K={K}, N={N}); fwd+dgrad+wgrad in fp64 numpy, including bf16->fp64 conversion")
+            f"(K={K}, N={N}); bf16 fwd+dgrad+wgrad and MXFP8 quantize+fwd+dgrad+wgrad in fp64 numpy, "
+            "including bf16->fp64 conversion")
     return flops, sec, threads, desc
 
 
@@ -236,8 +331,11 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     config = {"workload": f"{args.workload}: G={wl.G} K={wl.K} N={wl.N} rows={wl.rows}"
                           f"{' (output buffers ' + str(wl.out_rows) + ' rows)' if wl.out_rows > wl.rows else ''}, "
-                          f"split sizes as in the workload table, stacked bf16 weights{', bias' if wl.bias else ''}, "
-                          "fwd + dgrad + wgrad(accumulate into fp32 main_grad)",
+                          f"split sizes as in the workload table, stacked bf16 weights{', bias' if wl.bias else ''}; "
+                          "one step = offsets + bf16 fwd/dgrad/wgrad(accumulate into fp32 main_grad), then "
+                          "MXFP8 cast of x, W, dy (rowwise + columnwise) and MXFP8 fwd/dgrad/wgrad"
+                          + (" on the mxfp8_g8 splits (G=8, rows in multiples of 128)" if args.workload == "bf16_g8"
+                             else " on the same splits"),
               "l2": "no flush: every step streams > 3 GB of operands (W 0.9 GiB, dy 0.45 GiB, "
                     "main_grad 1.75 GiB), far larger than the 126 MB L2",
               "parallelism": f"replicas x{world}"}
@@ -245,7 +343,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        steps = max(1, min(args.steps, 3))
+        steps = max(1, min(args.steps, 2))
         samples = []
         for i in range(max(0, min(args.warmup, 1)) + steps):
             fl, sec, thr, desc = oracle_sample(args.workload)
@@ -269,7 +367,8 @@ def main():
     step = Step(args.workload, seed_offset=rank, device=dev)
     pk = peaks()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    nev = len(step.names) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
     sampler.start()  # sample clocks through warm-up and the timed region
     for _ in range(max(args.warmup, 3)):
@@ -293,40 +392,52 @@ def main():
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms_total = float(t.item())
     ms_step = ms_total / args.steps
-    status = int(step.status.item())
+    status = int(step.status.item()) | int(step.mx.status.item())
 
-    names = ["offsets", "fwd", "dgrad", "wgrad"]
     op_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
-             for j, n in enumerate(names)}
+             for j, n in enumerate(step.names)}
     timed_s = ms_total / 1e3
-    peak_tf = pk["bf16_tflops_sustained"] if timed_s > 1.0 else pk["bf16_tflops"]
-    peak_kind = "sustained" if timed_s > 1.0 else "burst"
+    sustained = timed_s > 1.0
+    peak_bf16 = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    peak_kind = "sustained" if sustained else "burst"
+    # MXFP8 tensor peak: the measured bf16 peak x 2 (dense fp8 / bf16 nominal ratio 4.5 / 2.25)
+    peak_of = {"bf16": peak_bf16, "mxfp8": 2.0 * peak_bf16}
     ops = {}
-    for n in names:
-        s = op_ms[n] / 1e3
-        if n == "offsets":
-            ops[n] = {"ms": op_ms[n], "gbs": step.bytes[n] / s / 1e9}
-            continue
-        tflops = step.flops / s / 1e12
-        t_roof = max(step.flops / (peak_tf * 1e12), step.bytes[n] / (pk["hbm_gbs"] * 1e9))
-        ops[n] = {"ms": op_ms[n], "tflops": tflops, "gbs": step.bytes[n] / s / 1e9,
-                  "frac_of_roofline": t_roof / s, "frac_of_bf16_peak": tflops / peak_tf}
-    dom = max(["fwd", "dgrad", "wgrad"], key=lambda n: op_ms[n])
-    dom_tf = ops[dom]["tflops"]
-    value = 3 * step.flops * world / (ms_step / 1e3) / 1e12
+    for n in step.names:
+        sec = op_ms[n] / 1e3
+        by = step.bytes[n]
+        fl = step.flops.get(n, 0.0)
+        e = {"ms": op_ms[n], "gbs": by / sec / 1e9}
+        if fl:
+            pkt = peak_of[step.dtype[n]]
+            t_roof = max(fl / (pkt * 1e12), by / (pk["hbm_gbs"] * 1e9))
+            e.update({"tflops": fl / sec / 1e12, "dtype": step.dtype[n], "peak_tflops": pkt,
+                      "frac_of_roofline": t_roof / sec, "frac_of_tensor_peak": fl / sec / 1e12 / pkt})
+        else:
+            e.update({"frac_of_hbm": by / sec / 1e9 / pk["hbm_gbs"]})
+        ops[n] = e
+    dom = max(step.names, key=lambda n: op_ms[n])
+    if step.flops.get(dom):
+        roof = {"bound": "tensor", "kernel": f"{dom}", "achieved": ops[dom]["tflops"],
+                "peak": peak_of[step.dtype[dom]], "unit": "TFLOP/s",
+                "frac": ops[dom]["tflops"] / peak_of[step.dtype[dom]],
+                "peak_source": f"{pk['source']} bf16 ({peak_kind})" + (" x2 for fp8" if step.dtype[dom] == "mxfp8" else ""),
+                "traffic": None}
+    else:
+        roof = {"bound": "hbm", "kernel": dom, "achieved": ops[dom]["gbs"], "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": ops[dom]["gbs"] / pk["hbm_gbs"],
+                "peak_source": f"{pk['source']} copy bandwidth", "traffic": None}
+    value = step.total_flops * world / (ms_step / 1e3) / 1e12
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config, "status_word": status,
-            "roofline": {"bound": "tensor", "kernel": f"grouped_gemm_kernel ({dom})", "achieved": dom_tf,
-                         "peak": peak_tf, "unit": "TFLOP/s", "frac": dom_tf / peak_tf,
-                         "peak_source": f"{pk['source']} bf16 ({peak_kind})", "traffic": None},
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16+mxfp8", "data": "synthetic",
+            "config": config, "status_word": status, "roofline": roof,
             "ops": ops, "gpu_launches": step.launches * args.steps, "clocks": clocks}
 
     if rank == 0:
         ms_e2e, h2d, d2h, st2 = e2e_measure(step, max(3, args.steps // 2), 2)
-        line["e2e"] = {"value": 3 * step.flops * world / (ms_e2e / 1e3) / 1e12, "unit": "TFLOP/s",
+        line["e2e"] = {"value": step.total_flops * world / (ms_e2e / 1e3) / 1e12, "unit": "TFLOP/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
         if world == 1 and not args.no_cpu_baseline:
             fl, sec, thr, desc = oracle_sample(args.workload)
