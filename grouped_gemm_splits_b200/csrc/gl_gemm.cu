@@ -343,7 +343,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem_base + buf * C::kTileN;
         bool ok = true;
         for (int kb = 0; kb < tl.num_kb; ++kb) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+          // On a ragged wgrad tail the peer zeroes rows of its stage before
+          // relaying; acquire at cluster scope so those writes are visible.
+          const bool peer_zeroed = CG == 2 && MODE == kWgrad && kb == tl.num_kb - 1 &&
+                                   static_cast<int>(tl.r1 - tl.r0) - kb * BK < BK;
+          const bool landed = peer_zeroed ? mbar_wait_acq_cluster(&full[stage], phase, abort_flag)
+                                          : mbar_wait(&full[stage], phase, abort_flag);
+          if (!__all_sync(0xffffffffu, landed)) {
             report_abort(abort_flag, p.status);
             ok = false;
             break;
@@ -412,15 +418,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          bool zeroed = false;
           if (MODE == kWgrad && kb == tl.num_kb - 1) {
             const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
             if (valid < BK) {
               uint8_t* sa = smem + stage * C::kStageBytes;
               zero_tail_rows<MODE, CG>(sa, sa + C::kABytes, valid, ((valid + 15) >> 4) * 16, lane);
+              zeroed = true;
             }
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&full[stage]), 0));
+          if (lane == 0) {
+            const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
+            if (zeroed) mbar_arrive_cluster_release(leader_full);  // the leader's MMA reads our zeroes
+            else        mbar_arrive_cluster(leader_full);
+          }
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
