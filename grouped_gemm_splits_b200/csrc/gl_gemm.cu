@@ -67,7 +67,7 @@ struct Cfg {
 struct GemmParams {
   CUtensorMap tmA;    // FWD x{K,M} box{64,128}; DGRAD dy{N,M} box{64,128}; WGRAD dy{N,M} box{64,64}
   CUtensorMap tmB;    // stacked W{K,N,G}: FWD box{64,BRows,1}, DGRAD box{64,64,1}; WGRAD x{K,M} box{64,64}
-  CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,128,1}
+  CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,32,1}
   const int64_t* offsets;  // G+1 entries
   int32_t* status;
   int64_t M;
@@ -442,7 +442,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================== epilogue (warps 2..5, both CTAs) =====================
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
-    const bool issuer = (warp == 2 && lane == 0);
     const uint32_t tempty_leader = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : 0u;
     int it = 0;
     int chunk_ctr = 0;
@@ -452,20 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tph = (it >> 1) & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
       if (!ok) report_abort(abort_flag, p.status);
-      if (MODE == kWgrad) {
-        // all four warps must agree before any named barrier below
-        uint32_t bad;
-        asm volatile(
-            "{\n\t.reg .pred P, Q;\n\t"
-            "setp.ne.b32 P, %1, 0;\n\t"
-            "bar.red.or.pred Q, 1, 128, P;\n\t"
-            "selp.b32 %0, 1, 0, Q;\n\t}"
-            : "=r"(bad)
-            : "r"((!ok || *abort_flag) ? 1 : 0));
-        if (bad) break;
-      } else if (!ok) {
-        break;
-      }
+      if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * C::kTileN + (static_cast<uint32_t>(q * 32) << 16);
       auto release_acc = [&]() {
@@ -522,17 +508,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // main_grad box: rows n0.. (TMEM lanes) x cols k0.. (TMEM columns)
-        float* staging = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
-        const int n0 = tl.mt * C::kTileM + hr;
+        // main_grad rows n0.. (this warp's 32 TMEM lanes) x cols k0 + 32c: each
+        // epilogue warp stages and stores its own [32 x 32] fp32 boxes
+        float* wstage = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes) + (warp - 2) * (2 * 32 * 32);
+        const int n0 = tl.mt * C::kTileM + hr + q * 32;
         const int k0 = tl.nt * C::kTileN;
         const int nchunks = min(C::kTileN / 32, ceil_div_i(p.K - k0, 32));
         const bool have_acc = tl.num_kb > 0;
         const bool rows_in = n0 < p.N;  // the pair's second half may lie past N
         for (int c = 0; c < nchunks; ++c, ++chunk_ctr) {
-          float* stg = staging + (chunk_ctr & 1) * (128 * 32);
-          if (issuer) bulk_wait_group_read<1>();  // the buffer's previous store has read it
-          named_barrier_sync(1, 128);
+          float* stg = wstage + (chunk_ctr & 1) * (32 * 32);
+          if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+          __syncwarp();
           uint32_t r[32];
           if (have_acc) {
             tmem_ld_32x32b_x32(tacc + c * 32, r);
@@ -542,16 +529,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) r[j] = 0u;
           }
           if (c == nchunks - 1) release_acc();
-          // row `row_in_tile` of a [128 x 32] fp32 box, 128-byte swizzle
-          uint8_t* rowp = reinterpret_cast<uint8_t*>(stg) + row_in_tile * 128;
+          // row `lane` of a [32 x 32] fp32 box, 128-byte swizzle
+          uint8_t* rowp = reinterpret_cast<uint8_t*>(stg) + lane * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int pj = j ^ (row_in_tile & 7);
+            const int pj = j ^ (lane & 7);
             *reinterpret_cast<uint4*>(rowp + pj * 16) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
           }
           fence_proxy_async_smem();
-          named_barrier_sync(1, 128);
-          if (issuer && rows_in) {
+          __syncwarp();
+          if (lane == 0 && rows_in) {
             const int kc = k0 + c * 32;
             if (PG) {
               if (p.accumulate) tma_reduce_add_2d(pg.map(tl.g), stg, kc, n0);
@@ -565,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (MODE == kWgrad && issuer) bulk_wait_group<0>();
+    if (MODE == kWgrad && lane == 0) bulk_wait_group<0>();  // stores of this warp done
   }
 
   tc_fence_before();
@@ -686,7 +673,7 @@ gl_status launch_mode(const GemmCall& c) {
     if (MODE == kFwd) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, BK, Cf::kBRows, BF, 2);
     if (MODE == kDgrad) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, 64, BK, BF, 2);
     if (MODE == kWgrad)
-      ok &= make_3d(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 32, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+      ok &= make_3d(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
     if (!ok) return GL_ERR_UNSUPPORTED;
     prm.offsets = c.offsets;
     prm.G = c.G;
@@ -717,7 +704,7 @@ gl_status launch_mode(const GemmCall& c) {
         const void* gp = (c.out_grouped.mode == GL_STACKED)
                              ? static_cast<const uint8_t*>(c.out_grouped.base) + static_cast<size_t>(g) * c.N * c.K * 4
                              : c.out_grouped.ptrs[g];
-        ok &= make_2d(&pga->tm[i], gp, c.K, c.N, 32, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+        ok &= make_2d(&pga->tm[i], gp, c.K, c.N, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
       }
     }
     if (!ok) { st = GL_ERR_UNSUPPORTED; break; }

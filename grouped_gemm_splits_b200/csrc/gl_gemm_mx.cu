@@ -32,7 +32,7 @@ namespace {
 constexpr int BK = 128;  // fp8 contraction elements per stage (128 bytes)
 constexpr int TM = 128;  // accumulator rows
 constexpr int TN = 224;  // accumulator columns
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // + warp 6: scale repacking
 constexpr int kPG = 64;
 constexpr int kBand = 8;
 constexpr int kSfCol0 = 2 * TN;  // first TMEM column of the scale-factor slots
@@ -55,6 +55,7 @@ struct CfgMX {
   static constexpr int kStagingBytes = (MODE == kWgrad) ? 2 * 128 * 32 * 4 : 0;
   static constexpr int kBarOffset = (kStagingOffset + kStagingBytes + 1023) / 1024 * 1024;
   static constexpr int kPrefixOffset = kBarOffset + 256;
+  static_assert((3 * kStages + 5) * 8 + 16 <= 256, "barrier area");
   // operand majorness in shared memory (1 = MN-major); SF source kind (1 = columnwise)
   static constexpr int kAMN = (MODE == kWgrad) ? 1 : 0;
   static constexpr int kBMN = (MODE == kFwd) ? 0 : 1;
@@ -67,7 +68,7 @@ struct MxParams {
   CUtensorMap tmB;    // stacked B codes: FWD W{K,N,G} box{128,224,1}; DGRAD Wc{K,N,G} box{128,128,1}; WGRAD x_c{K,M} box{128,128}
   CUtensorMap tmSA;   // A scales: FWD/DGRAD k-group words {pitchM, Kc/128} box{128,1}; WGRAD dy_sc{N,S} box{128,4}
   CUtensorMap tmSB;   // stacked B scales: FWD {pitchGN, K/128} box{224,1}; DGRAD Wsc{K,G*N32} box{224,4}; WGRAD x_sc{K,S} box{224,4}
-  CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,128,1}
+  CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,32,1}
   const int64_t* offsets;
   int32_t* status;
   int64_t out_rows;
@@ -186,7 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* empty = full + C::kStages;
-  uint64_t* tfull = empty + C::kStages;
+  uint64_t* sfready = empty + C::kStages;  // stage scales repacked (warp 6)
+  uint64_t* tfull = sfready + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -204,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sfready[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -323,7 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t d_tmem = tmem_base + buf * TN;
       bool ok = true;
       for (int kb = 0; kb < tl.num_kb; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+        // stage landed (TMA) and its scales repacked / tail rows zeroed (warp 6)
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag) &&
+                                         mbar_wait(&sfready[stage], phase, abort_flag))) {
           report_abort(abort_flag, p.status);
           ok = false;
           break;
@@ -334,29 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sf = smem + C::kSfOffset + stage * kSfStage;
         int ksteps = BK / 32;
         if (MODE == kWgrad && kb == tl.num_kb - 1) {
-          // ragged contraction: skip 32-row steps past the group's end and zero
-          // the code rows of the last partial step (A: one 128-column chunk,
-          // B: two; 128 bytes per row)
           const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
-          if (valid < BK) {
-            ksteps = (valid + 31) >> 5;
-            const int nrows = ksteps * 32 - valid;
-            const int per_chunk = nrows * 8;
-            for (int idx = lane; idx < 3 * per_chunk; idx += 32) {
-              const int chunk = idx / per_chunk;
-              const int rem = idx - chunk * per_chunk;
-              const int r = valid + (rem >> 3);
-              uint8_t* base = chunk == 0 ? sa : (sb + (chunk - 1) * 16384);
-              *reinterpret_cast<uint4*>(base + r * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
-            }
-          }
+          if (valid < BK) ksteps = (valid + 31) >> 5;
         }
-        // repack this stage's scales (A: 128 rows, B: 224 rows)
-        pack_scales<C::kSfaCol != 0>(sf, reinterpret_cast<uint32_t*>(sf + kPackA), TM, TM,
-                                     static_cast<int>(tl.r0 & 3), lane);
-        pack_scales<C::kSfbCol != 0>(sf + kRawB, reinterpret_cast<uint32_t*>(sf + kPackB), TN, TN, 0, lane);
-        fence_proxy_async_smem();
-        __syncwarp();
         if (lane == 0) {
           const uint32_t slot = tmem_base + kSfCol0 + stage * 16;
           const uint32_t sfa = slot, sfb = slot + 4;
@@ -390,11 +375,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_bounded(mma_done, 0);
     }
     __syncwarp();
+  } else if (warp == 6) {
+    // ===================== scale repack (and wgrad tail zeroing) =====================
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const Tile tl = decode<MODE>(t, prefix, p);
+      bool ok = true;
+      for (int kb = 0; kb < tl.num_kb; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+          report_abort(abort_flag, p.status);
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + stage * kOpStage;
+        uint8_t* sb = sa + C::kABytes;
+        uint8_t* sf = smem + C::kSfOffset + stage * kSfStage;
+        if (MODE == kWgrad && kb == tl.num_kb - 1) {
+          // ragged contraction: zero the code rows of the last partial 32-row
+          // MMA step (A: one 128-column chunk, B: two; 128 bytes per row); the
+          // MMA warp skips the steps past the group's end
+          const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
+          if (valid < BK) {
+            const int nrows = ((valid + 31) >> 5) * 32 - valid;
+            const int per_chunk = nrows * 8;
+            for (int idx = lane; idx < 3 * per_chunk; idx += 32) {
+              const int chunk = idx / per_chunk;
+              const int rem = idx - chunk * per_chunk;
+              const int r = valid + (rem >> 3);
+              uint8_t* base = chunk == 0 ? sa : (sb + (chunk - 1) * 16384);
+              *reinterpret_cast<uint4*>(base + r * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+            }
+          }
+        }
+        pack_scales<C::kSfaCol != 0>(sf, reinterpret_cast<uint32_t*>(sf + kPackA), TM, TM,
+                                     static_cast<int>(tl.r0 & 3), lane);
+        pack_scales<C::kSfbCol != 0>(sf + kRawB, reinterpret_cast<uint32_t*>(sf + kPackB), TN, TN, 0, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfready[stage]);
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
   } else {
     // ===================== epilogue =====================
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
-    const bool issuer = (warp == 2 && lane == 0);
     int it = 0;
     int chunk_ctr = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
@@ -403,19 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tph = (it >> 1) & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
       if (!ok) report_abort(abort_flag, p.status);
-      if (MODE == kWgrad) {
-        uint32_t bad;
-        asm volatile(
-            "{\n\t.reg .pred P, Q;\n\t"
-            "setp.ne.b32 P, %1, 0;\n\t"
-            "bar.red.or.pred Q, 1, 128, P;\n\t"
-            "selp.b32 %0, 1, 0, Q;\n\t}"
-            : "=r"(bad)
-            : "r"((!ok || *abort_flag) ? 1 : 0));
-        if (bad) break;
-      } else if (!ok) {
-        break;
-      }
+      if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * TN + (static_cast<uint32_t>(q * 32) << 16);
       auto release_acc = [&]() {
@@ -467,15 +482,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        float* staging = reinterpret_cast<float*>(smem + C::kStagingOffset);
-        const int n0 = tl.mt * TM;
+        // main_grad rows n0.. (this warp's 32 TMEM lanes) x cols k0 + 32c: each
+        // epilogue warp stages and stores its own [32 x 32] fp32 boxes
+        float* wstage = reinterpret_cast<float*>(smem + C::kStagingOffset) + (warp - 2) * (2 * 32 * 32);
+        const int n0 = tl.mt * TM + q * 32;
         const int k0 = tl.nt * TN;
         const int nchunks = min(TN / 32, cdiv(p.K - k0, 32));
         const bool have_acc = tl.num_kb > 0;
+        const bool rows_in = n0 < p.N;
         for (int c = 0; c < nchunks; ++c, ++chunk_ctr) {
-          float* stg = staging + (chunk_ctr & 1) * (128 * 32);
-          if (issuer) bulk_wait_group_read<1>();
-          named_barrier_sync(1, 128);
+          float* stg = wstage + (chunk_ctr & 1) * (32 * 32);
+          if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+          __syncwarp();
           uint32_t r[32];
           if (have_acc) {
             tmem_ld_32x32b_x32(tacc + c * 32, r);
@@ -485,15 +503,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) r[j] = 0u;
           }
           if (c == nchunks - 1) release_acc();
-          uint8_t* rowp = reinterpret_cast<uint8_t*>(stg) + row_in_tile * 128;
+          // row `lane` of a [32 x 32] fp32 box, 128-byte swizzle
+          uint8_t* rowp = reinterpret_cast<uint8_t*>(stg) + lane * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int pj = j ^ (row_in_tile & 7);
+            const int pj = j ^ (lane & 7);
             *reinterpret_cast<uint4*>(rowp + pj * 16) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
           }
           fence_proxy_async_smem();
-          named_barrier_sync(1, 128);
-          if (issuer) {
+          __syncwarp();
+          if (lane == 0 && rows_in) {
             const int kc = k0 + c * 32;
             if (PG) {
               if (p.accumulate) tma_reduce_add_2d(pg.map(tl.g), stg, kc, n0);
@@ -507,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (MODE == kWgrad && issuer) bulk_wait_group<0>();
+    if (MODE == kWgrad && lane == 0) bulk_wait_group<0>();  // stores of this warp done
   }
 
   tc_fence_before();
@@ -598,7 +617,7 @@ gl_status mx_mode(const MxCall& c) {
       ok &= map3(&prm.tmB, c.w.base, c.K, c.N, c.G, 1, 128, 128, U8);
       ok &= map2(&prm.tmSB, c.ws.base, c.K, static_cast<uint64_t>(c.G) * prm.n32, c.K, TN, 4, U8, NOSW);
     } else {
-      ok &= map3(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 4, 32, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+      ok &= map3(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
     }
     if (!ok) return GL_ERR_UNSUPPORTED;
     prm.offsets = c.offsets;
@@ -616,7 +635,7 @@ gl_status mx_mode(const MxCall& c) {
       const int g = g0 + i;
       if (MODE == kWgrad) {
         const void* gp = group_ptr(c.out_grouped, g, static_cast<size_t>(c.N) * c.K * 4);
-        ok &= map2(&pga->tm[i], gp, c.K, c.N, static_cast<uint64_t>(c.K) * 4, 32, 128,
+        ok &= map2(&pga->tm[i], gp, c.K, c.N, static_cast<uint64_t>(c.K) * 4, 32, 32,
                    CU_TENSOR_MAP_DATA_TYPE_FLOAT32, SW);
         continue;
       }
