@@ -53,7 +53,7 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return lo | (hi << 16);
 }
 
-__global__ void __launch_bounds__(kQThreads)
+__global__ void __launch_bounds__(kQThreads, 4)
     quantize_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int cols,
                     const int64_t* __restrict__ row_offsets, int G, const int32_t* __restrict__ status,
                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r,
@@ -98,11 +98,11 @@ __global__ void __launch_bounds__(kQThreads)
   const int c8 = lane;         // 8-column chunk within the 256-column tile
   const int rbase = warp * 4;  // this thread's 4 rows within the 32-row block
 
-  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+  // Where tile t lives: group g, block j, first row r0 and valid row count.
+  auto locate = [&](int64_t t, int& g, int64_t& j, int64_t& r0, int& vrows, int& cc) {
     const int64_t rb = t / ncc;
-    const int cc = static_cast<int>(t - rb * ncc);
-    int g;
-    int64_t j, gstart, gend;
+    cc = static_cast<int>(t - rb * ncc);
+    int64_t gstart, gend;
     if (row_offsets != nullptr) {
       int lo = 0, hi = G;
       while (hi - lo > 1) {
@@ -119,25 +119,48 @@ __global__ void __launch_bounds__(kQThreads)
       gstart = static_cast<int64_t>(g) * per;
       gend = gstart + per;
     }
-    const int64_t r0 = gstart + j * kQRows;
-    const int vrows = static_cast<int>(max(int64_t(0), min(static_cast<int64_t>(kQRows), gend - r0)));
+    r0 = gstart + j * kQRows;
+    vrows = static_cast<int>(max(int64_t(0), min(static_cast<int64_t>(kQRows), gend - r0)));
+  };
+  // 16-byte loads of this thread's 4 rows x 8 columns of tile t (zeros outside)
+  auto fetch = [&](int64_t r0, int vrows, int cc, uint4 (&raw)[4]) {
     const int col = cc * kQCols + c8 * 8;
-    const bool col_ok = col < cols;
-
-    // load 4 rows x 8 columns
-    float v[4][8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = rbase + i;
-      if (col_ok && r < vrows) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + (r0 + r) * cols + col));
-        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+      if (col < cols && r < vrows)
+        raw[i] = __ldg(reinterpret_cast<const uint4*>(src + (r0 + r) * cols + col));
+      else
+        raw[i] = make_uint4(0, 0, 0, 0);
+    }
+  };
+
+  int64_t t = blockIdx.x;
+  int g = 0, vrows = 0, cc = 0;
+  int64_t j = 0, r0 = 0;
+  uint4 raw[4];
+  if (t < ntiles) {
+    locate(t, g, j, r0, vrows, cc);
+    fetch(r0, vrows, cc, raw);
+  }
+  for (; t < ntiles; t += gridDim.x) {
+    // issue the next tile's loads before working on this one
+    const int64_t tn = t + gridDim.x;
+    int gn = 0, vrows_n = 0, cc_n = 0;
+    int64_t jn = 0, r0n = 0;
+    uint4 raw_n[4];
+    if (tn < ntiles) {
+      locate(tn, gn, jn, r0n, vrows_n, cc_n);
+      fetch(r0n, vrows_n, cc_n, raw_n);
+    }
+    const int col = cc * kQCols + c8 * 8;
+    const bool col_ok = col < cols;
+    float v[4][8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[i][k] = __bfloat162float(h[k]);
-      } else {
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw[i]);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[i][k] = 0.0f;
-      }
+      for (int k = 0; k < 8; ++k) v[i][k] = __bfloat162float(h[k]);
     }
 
     if (codes_r != nullptr) {
@@ -207,6 +230,13 @@ __global__ void __launch_bounds__(kQThreads)
       }
       __syncthreads();  // cmax / csf are reused by the next tile
     }
+    g = gn;
+    j = jn;
+    r0 = r0n;
+    vrows = vrows_n;
+    cc = cc_n;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) raw[i] = raw_n[i];
   }
 }
 
@@ -218,7 +248,7 @@ gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t
   const int smem = row_offsets != nullptr ? (G + 1) * static_cast<int>(sizeof(int64_t)) : 0;
   if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel), smem + 16 * 1024) != cudaSuccess)
     return GL_ERR_CUDA;
-  const int grid = num_sms() * 8;
+  const int grid = num_sms() * 4;
   quantize_kernel<<<grid, kQThreads, smem, stream>>>(
       static_cast<const __nv_bfloat16*>(src), rows, cols, row_offsets, G, status, codes_r,
       scales_r, codes_c, scales_c, scale_layout == GL_SCALES_KGROUP ? static_cast<int>((rows + 3) / 4 * 4) : 0);
