@@ -205,6 +205,7 @@ gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_group
   c.M = M;
   c.N = N;
   c.K = K;
+  c.cta_pair = g_cta_pair.load();
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
@@ -237,6 +238,7 @@ gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_g
   c.M = M;
   c.N = N;
   c.K = K;
+  c.cta_pair = g_cta_pair.load();
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
@@ -273,6 +275,7 @@ gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, co
   c.N = N;
   c.K = K;
   c.accumulate = accumulate ? 1 : 0;
+  c.cta_pair = g_cta_pair.load();
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }

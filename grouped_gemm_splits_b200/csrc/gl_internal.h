@@ -64,6 +64,7 @@ struct MxCall {
   int64_t M;
   int N, K;
   int accumulate;
+  int cta_pair;  // 1: 256x224 tiles on CTA pairs; 0: 128x224 tiles per CTA
   cudaStream_t stream;
 };
 

@@ -83,10 +83,11 @@ const char* gl_status_string(gl_status s);
 
 /*
  * gl_set_cta_pair -- tile shape of the grouped GEMMs launched afterwards by
- * this process: enable != 0 (the default) computes 256 x 256 output tiles on
- * pairs of CTAs (tcgen05 cta_group::2, one CTA per SM); enable == 0 computes
- * 128 x 256 tiles on single CTAs.  Results agree within rounding; the pair
- * shape moves less operand data per flop.  Always returns GL_OK.
+ * this process: enable != 0 (the default) computes 256-row output tiles on
+ * pairs of CTAs (tcgen05 cta_group::2, one CTA per SM; 256 x 256 for bf16,
+ * 256 x 224 for MXFP8); enable == 0 computes 128-row tiles on single CTAs.
+ * Results agree within rounding; the pair shape moves less operand data per
+ * flop.  Always returns GL_OK.
  */
 gl_status gl_set_cta_pair(int enable);
 

@@ -18,6 +18,14 @@ from tests.gpu_util import f64, offsets_on_device, sample_rows, sentinel_like, u
 
 pytestmark = pytest.mark.gpu
 
+
+@pytest.fixture(params=["pair", "single"])
+def tile_mode(request):
+    """Run with 256-row tiles on CTA pairs and with 128-row tiles on single CTAs."""
+    gl.gl_set_cta_pair(request.param == "pair")
+    yield request.param
+    gl.gl_set_cta_pair(True)
+
 TOL_MX = 1e-2
 
 
@@ -57,7 +65,7 @@ SMALL = [
 
 @pytest.mark.parametrize("G,N,K,m", SMALL)
 @pytest.mark.parametrize("per_group", [False, True])
-def test_mxfp8_small(G, N, K, m, per_group):
+def test_mxfp8_small(G, N, K, m, per_group, tile_mode):
     M = int(sum(m))
     d = {k: v.cuda() for k, v in synth.operands(G, M, N, K, seed=G + N + K, bias=True).items()}
     off, st = offsets_on_device(m, M, M + 32)
@@ -107,7 +115,7 @@ def test_mxfp8_small(G, N, K, m, per_group):
     assert untouched(y[M:]) and untouched(dx[M:])
 
 
-def test_mxfp8_integer_mode_bit_exact():
+def test_mxfp8_integer_mode_bit_exact(tile_mode):
     """Values in {-1,0,1}: every block scales by 2^-8 (or is all zero), the
     codes are exact, and every product sum is an exact small integer."""
     G, N, K, m = 3, 256, 128, [0, 100, 156]
@@ -129,7 +137,7 @@ def test_mxfp8_integer_mode_bit_exact():
     assert np.array_equal(f64(mg), orc.wgrad(x64, dy64, m, f64(d["main_grad"]), True))
 
 
-def test_mxfp8_full_size_sampled():
+def test_mxfp8_full_size_sampled(tile_mode):
     """The MXFP8 workload (G=8, K=4096, N=14336, 16384 rows in multiples of
     128) at full size; sampled entries against the oracle, which quantizes
     exactly the rows / columns each entry needs."""
