@@ -6,7 +6,10 @@
 
 namespace {
 
-std::atomic<int> g_cta_pair{1};
+// bit 0: bf16 GEMMs on CTA pairs (default on); bit 1: MXFP8 GEMMs on CTA
+// pairs (default off: their per-stage cross-CTA hand-off of repacked scales
+// needs cluster-scope ordering, which costs more than the pair tile saves).
+std::atomic<int> g_cta_pair{GL_PAIRS_BF16};
 
 using gl::GemmCall;
 
@@ -61,8 +64,9 @@ const char* gl_status_string(gl_status s) {
   return "unknown status";
 }
 
-gl_status gl_set_cta_pair(int enable) {
-  g_cta_pair.store(enable ? 1 : 0);
+gl_status gl_set_cta_pair(int flags) {
+  if (flags & ~(GL_PAIRS_BF16 | GL_PAIRS_MXFP8)) return GL_ERR_INVALID;
+  g_cta_pair.store(flags);
   return GL_OK;
 }
 
@@ -98,7 +102,7 @@ gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int6
   c.M = M;
   c.N = N;
   c.K = K;
-  c.cta_pair = g_cta_pair.load();
+  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_BF16) ? 1 : 0;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -125,7 +129,7 @@ gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t
   c.M = M;
   c.N = N;
   c.K = K;
-  c.cta_pair = g_cta_pair.load();
+  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_BF16) ? 1 : 0;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -158,7 +162,7 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
   c.N = N;
   c.K = K;
   c.accumulate = accumulate ? 1 : 0;
-  c.cta_pair = g_cta_pair.load();
+  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_BF16) ? 1 : 0;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -205,7 +209,7 @@ gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_group
   c.M = M;
   c.N = N;
   c.K = K;
-  c.cta_pair = g_cta_pair.load();
+  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_MXFP8) ? 1 : 0;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
@@ -238,7 +242,7 @@ gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_g
   c.M = M;
   c.N = N;
   c.K = K;
-  c.cta_pair = g_cta_pair.load();
+  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_MXFP8) ? 1 : 0;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
@@ -275,7 +279,7 @@ gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, co
   c.N = N;
   c.K = K;
   c.accumulate = accumulate ? 1 : 0;
-  c.cta_pair = g_cta_pair.load();
+  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_MXFP8) ? 1 : 0;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }

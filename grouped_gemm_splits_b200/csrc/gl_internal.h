@@ -5,7 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/gl.h"
+#include "gl.h"
 
 namespace gl {
 

@@ -108,9 +108,14 @@ def _shape_nk(w: TensorOrList):
     return tuple((w if isinstance(w, torch.Tensor) else w[0]).shape[-2:])
 
 
-def gl_set_cta_pair(enable: bool) -> None:
-    """Tile shape of later GEMM launches: CTA pairs (256x256, default) or single CTAs (128x256)."""
-    _check(load().gl_set_cta_pair(1 if enable else 0), "gl_set_cta_pair")
+GL_PAIRS_BF16, GL_PAIRS_MXFP8 = 1, 2
+
+
+def gl_set_cta_pair(bf16: bool = True, mxfp8: bool = False) -> None:
+    """Tile shape of later GEMM launches: CTA pairs (256-row tiles) or single
+    CTAs (128-row tiles), separately for the bf16 and the MXFP8 GEMMs."""
+    _check(load().gl_set_cta_pair((GL_PAIRS_BF16 if bf16 else 0) | (GL_PAIRS_MXFP8 if mxfp8 else 0)),
+           "gl_set_cta_pair")
 
 
 def gl_offsets(m_splits: torch.Tensor, expect_rows: int, out_rows: Optional[int] = None,

@@ -83,13 +83,16 @@ const char* gl_status_string(gl_status s);
 
 /*
  * gl_set_cta_pair -- tile shape of the grouped GEMMs launched afterwards by
- * this process: enable != 0 (the default) computes 256-row output tiles on
- * pairs of CTAs (tcgen05 cta_group::2, one CTA per SM; 256 x 256 for bf16,
- * 256 x 224 for MXFP8); enable == 0 computes 128-row tiles on single CTAs.
- * Results agree within rounding; the pair shape moves less operand data per
- * flop.  Always returns GL_OK.
+ * this process.  With GL_PAIRS_BF16 set (default) the bf16 GEMMs compute
+ * 256 x 256 output tiles on pairs of CTAs (tcgen05 cta_group::2, one CTA per
+ * SM), else 128 x 256 tiles on single CTAs.  With GL_PAIRS_MXFP8 set the
+ * MXFP8 GEMMs compute 256 x 224 tiles on CTA pairs, else (default) 128 x 224
+ * tiles on single CTAs.  Results agree within rounding.  Returns
+ * GL_ERR_INVALID for unknown flag bits.
  */
-gl_status gl_set_cta_pair(int enable);
+#define GL_PAIRS_BF16 1
+#define GL_PAIRS_MXFP8 2
+gl_status gl_set_cta_pair(int flags);
 
 /*
  * gl_offsets -- group row offsets from the split sizes, on the device.

@@ -23,9 +23,9 @@ pytestmark = pytest.mark.gpu
 def tile_mode(request):
     """Run a test with 256x256 tiles on CTA pairs and with 128x256 tiles on
     single CTAs; the default (pairs) is restored afterwards."""
-    gl.gl_set_cta_pair(request.param == "pair")
+    gl.gl_set_cta_pair(bf16=request.param == "pair")
     yield request.param
-    gl.gl_set_cta_pair(True)
+    gl.gl_set_cta_pair()  # defaults
 
 # (G, N, K, m_splits): several tiles, ragged tails in every dimension,
 # empty groups, groups shorter than one MMA step.

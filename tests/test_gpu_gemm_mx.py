@@ -22,9 +22,9 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(params=["pair", "single"])
 def tile_mode(request):
     """Run with 256-row tiles on CTA pairs and with 128-row tiles on single CTAs."""
-    gl.gl_set_cta_pair(request.param == "pair")
+    gl.gl_set_cta_pair(mxfp8=request.param == "pair")
     yield request.param
-    gl.gl_set_cta_pair(True)
+    gl.gl_set_cta_pair()  # defaults
 
 TOL_MX = 1e-2
 
