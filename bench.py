@@ -35,6 +35,15 @@ METRIC = "grouped-GEMM TFLOPS fwd/dgrad/wgrad and % of B200 dense BF16/MXFP8 pea
 WORKLOAD = "bf16_g8"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per launch from one ncu capture of the current
+# kernels at the bench workload (profiles/step_bf16_g8_launch_list.md); an
+# entry must be removed when its kernel changes.
+MEASURED_TRAFFIC = {
+    "bf16_g8": {"fwd": 2916439040, "dgrad": 4142550528, "wgrad": 5272824832,
+                "quant_x": 219281664, "quant_w": 1860770304, "quant_dy": 904451584,
+                "fwd_mx": 1309727232, "dgrad_mx": 1649219072, "wgrad_mx": 3573024512},
+}
+
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -408,6 +417,10 @@ def main():
         by = step.bytes[n]
         fl = step.flops.get(n, 0.0)
         e = {"ms": op_ms[n], "gbs": by / sec / 1e9}
+        tr = MEASURED_TRAFFIC.get(args.workload, {}).get(n)
+        if tr:
+            e["dram_traffic_bytes"] = tr
+            e["traffic_over_algorithmic"] = tr / by
         if fl:
             pkt = peak_of[step.dtype[n]]
             t_roof = max(fl / (pkt * 1e12), by / (pk["hbm_gbs"] * 1e9))
@@ -422,11 +435,12 @@ def main():
                 "peak": peak_of[step.dtype[dom]], "unit": "TFLOP/s",
                 "frac": ops[dom]["tflops"] / peak_of[step.dtype[dom]],
                 "peak_source": f"{pk['source']} bf16 ({peak_kind})" + (" x2 for fp8" if step.dtype[dom] == "mxfp8" else ""),
-                "traffic": None}
+                "traffic": MEASURED_TRAFFIC.get(args.workload, {}).get(dom)}
     else:
         roof = {"bound": "hbm", "kernel": dom, "achieved": ops[dom]["gbs"], "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": ops[dom]["gbs"] / pk["hbm_gbs"],
-                "peak_source": f"{pk['source']} copy bandwidth", "traffic": None}
+                "peak_source": f"{pk['source']} copy bandwidth",
+                "traffic": MEASURED_TRAFFIC.get(args.workload, {}).get(dom)}
     value = step.total_flops * world / (ms_step / 1e3) / 1e12
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
