@@ -39,9 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernels at the bench workload (profiles/step_bf16_g8_launch_list.md); an
 # entry must be removed when its kernel changes.
 MEASURED_TRAFFIC = {
-    "bf16_g8": {"fwd": 2916439040, "dgrad": 4142550528, "wgrad": 5272824832,
-                "quant_x": 219281664, "quant_w": 1860770304, "quant_dy": 904451584,
-                "fwd_mx": 1309727232, "dgrad_mx": 1649219072, "wgrad_mx": 3573024512},
+    "bf16_g8": {"fwd": 2916439040, "dgrad": 4142550528, "wgrad": 5272824832},
 }
 
 
@@ -159,14 +157,14 @@ class MxStep:
             ev[i0].record()
         gl.gl_offsets(self.m_dev, wl.rows, wl.rows, self.offsets, self.status)
         gl.group_quantize_mxfp8(self.x, self.offsets, rowwise=True, colwise=True, status=self.status,
-                                out=self.qx, kgroup_scales=True)
+                                out=self.qx, mma_scales=True)
         if ev:
             ev[i0 + 1].record()
-        gl.group_quantize_mxfp8(self.w, rowwise=True, colwise=True, out=self.qw, kgroup_scales=True)
+        gl.group_quantize_mxfp8(self.w, rowwise=True, colwise=True, out=self.qw, mma_scales=True)
         if ev:
             ev[i0 + 2].record()
         gl.group_quantize_mxfp8(self.dy, self.offsets, rowwise=True, colwise=True, status=self.status,
-                                out=self.qdy, kgroup_scales=True)
+                                out=self.qdy, mma_scales=True)
         if ev:
             ev[i0 + 3].record()
         gl.gl_fwd_mxfp8(self.qx["codes_r"], self.qx["scales_r"], self.qw["codes_r"].view(G, N, K),

@@ -6,10 +6,9 @@
 
 namespace {
 
-// bit 0: bf16 GEMMs on CTA pairs (default on); bit 1: MXFP8 GEMMs on CTA
-// pairs (default off: their per-stage cross-CTA hand-off of repacked scales
-// needs cluster-scope ordering, which costs more than the pair tile saves).
-std::atomic<int> g_cta_pair{GL_PAIRS_BF16};
+// bit 0: bf16 GEMMs on CTA pairs; bit 1: MXFP8 GEMMs on CTA pairs (both on
+// by default).
+std::atomic<int> g_cta_pair{GL_PAIRS_BF16 | GL_PAIRS_MXFP8};
 
 using gl::GemmCall;
 
@@ -293,8 +292,8 @@ gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const in
   if (codes_r != nullptr && scales_r == nullptr) return GL_ERR_INVALID;
   if (codes_c != nullptr && scales_c == nullptr) return GL_ERR_INVALID;
   if (cols % 32 != 0) return GL_ERR_UNSUPPORTED;
-  if (scale_layout != GL_SCALES_ROWMAJOR && scale_layout != GL_SCALES_KGROUP) return GL_ERR_INVALID;
-  if (scale_layout == GL_SCALES_KGROUP && cols % 128 != 0) return GL_ERR_UNSUPPORTED;
+  if (scale_layout != GL_SCALES_ROWMAJOR && scale_layout != GL_SCALES_MMA) return GL_ERR_INVALID;
+  if (scale_layout == GL_SCALES_MMA && cols % 128 != 0) return GL_ERR_UNSUPPORTED;
   if (rows >= (int64_t(1) << 31)) return GL_ERR_UNSUPPORTED;
   if (row_offsets == nullptr && rows % G != 0) return GL_ERR_INVALID;
   if (!aligned16(src) || (codes_r && (reinterpret_cast<uintptr_t>(codes_r) & 7u)) ||
@@ -303,6 +302,14 @@ gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const in
   if (rows == 0) return GL_OK;
   return gl::launch_quantize(src, rows, cols, row_offsets, G, status, codes_r, scales_r, codes_c,
                              scales_c, scale_layout, to_stream(stream));
+}
+
+size_t gl_mxfp8_scale_bytes(int64_t rows, int cols, int G, int colwise, int scale_layout) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0 || G <= 0) return 0;
+  const size_t r = static_cast<size_t>(rows), c = static_cast<size_t>(cols), g = static_cast<size_t>(G);
+  if (scale_layout == GL_SCALES_ROWMAJOR) return colwise ? ((r + 31) / 32 + g) * c : r * (c / 32);
+  if (scale_layout != GL_SCALES_MMA || cols % 128 != 0) return 0;
+  return (colwise ? (r + 127) / 128 + g : (r + 127) / 128) * (c / 128) * 512;
 }
 
 }  // extern "C"

@@ -7,21 +7,30 @@
 // columnwise for wgrad), computed as sum_k (q_a 2^sa)(q_b 2^sb) by
 // tcgen05.mma kind::mxf8f6f4.block_scale with fp32 accumulation in TMEM.
 //
-// Output tile 128*CG x 224.  With CG = 2 a cluster pair shares the tile
-// (tcgen05 cta_group::2): each CTA loads its own 128 rows of A and 112 rows
-// of B; the leader issues the MMAs.  Two 224-column fp32 accumulators
-// (448 TMEM columns) leave 64 columns for per-stage scale-factor slots.
+// Output tile 128*CG x 192.  With CG = 2 a cluster pair shares the tile
+// (tcgen05 cta_group::2): each CTA loads its own 128 rows of A and 96 rows
+// of B; the peer relays "stage landed" to the leader, which issues the MMAs.
+// Two 192-column fp32 accumulators (384 TMEM columns) leave 128 columns for
+// the scale-factor slots.
 //
 // Per stage (128 contraction elements = four MMAs of K=32) the producer
-// TMA-loads the codes (128-byte swizzle) and the raw scales of the stage.
-// A repack warp turns the raw scales into the 32-row x 16-byte blocks that
-// tcgen05.cp.32x128b.warpx4 copies to TMEM (row i of a 128-row block at byte
-// (i%32)*16 + ((i/32)%4)*4 + kb) -- each CTA packs the scales of its own A
-// rows and of all 224 B rows -- and zeroes the rows of a ragged wgrad tail.
-// The MMA warp then copies the scales to TMEM and issues the four MMAs,
-// selecting scale byte kb of each MMA through the instruction descriptor.
-// Rowwise scales arrive k-group-major ([cols/128][rows] words of four
-// scales), columnwise scales as [blocks][cols] rows: one TMA box per stage.
+// TMA-loads the codes (128-byte swizzle) and the scales.  The scales arrive
+// from the quantizer in 512-byte atoms that already have the tcgen05
+// scale-factor layout (128 operand rows x 4 blocks; row i at byte
+// (i%32)*16 + ((i/32)%4)*4 + block), so a stage's scales are two plain boxes:
+// one atom for the CTA's 128 A rows and two consecutive atoms (256 rows)
+// covering the tile's 192 B rows.  The MMA thread copies them to TMEM with
+// tcgen05.cp.32x128b.warpx4 and selects scale byte kb of each MMA through the
+// instruction descriptor.  B row i of a tile that starts at operand row
+// 128c + 32s reads TMEM column (slot + s) + i/32, so the MMA's scale address is
+// offset by s columns; with 192-row tiles s is 0 or 2 (tiles start on
+// multiples of 64 rows).  A tiles (fprop / dgrad) start on 128-row boundaries of
+// the packed activations: a group's first tile may begin inside the previous
+// group, and only the group's own rows are stored.
+//
+// The only generic shared-memory writes on the main loop are the zeroed rows
+// of a ragged wgrad contraction tail (once per tile); on a pair the peer
+// publishes them with a cluster-scope release that the leader acquires.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -36,58 +45,58 @@ namespace gl {
 namespace {
 
 constexpr int BK = 128;  // fp8 contraction elements per stage (128 bytes)
-constexpr int TN = 224;  // accumulator columns
-constexpr int kThreads = 224;  // warp 0 TMA, 1 MMA, 2-5 epilogue, 6 scale repack
+constexpr int TN = 192;  // accumulator columns (tile starts on multiples of 64 B rows)
+constexpr int kThreads = 192;  // warp 0 TMA, 1 MMA (leader) / relay (peer), 2-5 epilogue
 constexpr int kPG = 64;
 constexpr int kBand = 8;
 constexpr int kSfCol0 = 2 * TN;  // first TMEM column of the scale-factor slots
-constexpr int kSfStage = 3072;   // raw A [0,528) | raw B [640,1536) | packed A 512 | packed B 1024
-constexpr int kRawB = 640, kPackA = 1536, kPackB = 2048;
+constexpr int kSfSlots = 4;      // slot j: A at +0 (4 columns), B at +4 (8 columns)
+constexpr int kSfSlotCols = 16;
+constexpr int kSfABytes = 512;   // one atom
+constexpr int kAtomsB = 2;       // 256 B rows cover a 192-row tile starting 0 or 64 rows into an atom
+constexpr int kSfBytes = 2048;   // A atom + B atoms, padded to keep stages 1 KB aligned
+static_assert(kSfABytes + kAtomsB * 512 <= kSfBytes, "scale staging");
+static_assert((TN % 64) == 0 && 64 + TN <= 128 * kAtomsB, "B tile must stay inside the loaded atoms");
 
 template <int MODE, int CG>
 struct CfgMX {
   static constexpr int kTileM = 128 * CG;
-  static constexpr int kBRows = TN / CG;  // B rows held per CTA (224 or 112)
+  static constexpr int kBRows = TN / CG;  // B rows held per CTA (192 or 96)
   static constexpr int kABytes = 128 * BK;  // 16 KB
   // B codes per CTA: K-major kBRows x 128 B, MN-major 128-column chunks
-  static constexpr int kBLoad = (MODE == kFwd) ? kBRows * BK : (CG == 1 ? 2 : 1) * 128 * BK;
-  static constexpr int kOpStage = kABytes + (CG == 1 ? 2 : 1) * 128 * BK;  // 48 KB / 32 KB
-  static constexpr int kStages = CG == 2 ? 5 : ((MODE == kWgrad) ? 3 : 4);
-  static constexpr int kSfSlot = CG == 2 ? 12 : 16;  // TMEM columns per stage slot
-  // rowwise A scales: 132 words from a 4-aligned row (TMA's first coordinate
-  // must be 16-byte aligned); columnwise: 4 rows x 128 bytes
-  static constexpr int kRawABytes = (MODE == kWgrad) ? 4 * 128 : (128 + 4) * 4;
-  static constexpr int kRawBBytes = TN * 4;  // 896 either way
-  static constexpr int kTx = kABytes + kBLoad + kRawABytes + kRawBBytes;
-  static constexpr int kSfOffset = kStages * kOpStage;
-  static constexpr int kStagingOffset = kSfOffset + kStages * kSfStage;
+  static constexpr int kBChunks = (CG == 1 ? 2 : 1);
+  static constexpr int kBAlloc = kBChunks * 128 * BK;
+  static constexpr int kBLoad = (MODE == kFwd) ? kBRows * BK : kBAlloc;
+  static constexpr int kStageBytes = kABytes + kBAlloc + kSfBytes;  // 50 KB / 34 KB
   static constexpr int kStagingBytes = (MODE == kWgrad) ? 4 * 2 * 32 * 32 * 4 : 0;
+  static constexpr int kStages = CG == 2 ? ((MODE == kWgrad) ? 5 : 6) : ((MODE == kWgrad) ? 3 : 4);
+  static constexpr int kTx = kABytes + kBLoad + kSfABytes + kAtomsB * 512;
+  static constexpr int kStagingOffset = kStages * kStageBytes;
   static constexpr int kBarOffset = (kStagingOffset + kStagingBytes + 1023) / 1024 * 1024;
   static constexpr int kPrefixOffset = kBarOffset + 256;
-  static_assert((3 * kStages + 5) * 8 + 16 <= 256, "barrier area");
-  static_assert(kSfCol0 + kStages * kSfSlot <= 512, "TMEM columns");
-  static_assert(kOpStage % 1024 == 0 && kSfOffset % 1024 == 0 && kStagingOffset % 1024 == 0, "alignment");
-  // operand majorness in shared memory (1 = MN-major); scale source kind (1 = columnwise)
+  static_assert((2 * kStages + 5) * 8 + 16 <= 256, "barrier area");
+  static_assert(kSfCol0 + kSfSlots * kSfSlotCols <= 512, "TMEM columns");
+  static_assert(kStageBytes % 1024 == 0 && kStagingOffset % 1024 == 0, "alignment");
+  // operand majorness in shared memory (1 = MN-major)
   static constexpr int kAMN = (MODE == kWgrad) ? 1 : 0;
   static constexpr int kBMN = (MODE == kFwd) ? 0 : 1;
-  static constexpr int kSfaCol = (MODE == kWgrad) ? 1 : 0;
-  static constexpr int kSfbCol = (MODE == kFwd) ? 0 : 1;
 };
 
 struct MxParams {
   CUtensorMap tmA;    // A codes: FWD x{K,M} / DGRAD dy{N,M} box{128,128}; WGRAD dy_c{N,M} box{128,128}
   CUtensorMap tmB;    // stacked B codes: FWD W{K,N,G} box{128,BRows,1}; DGRAD Wc{K,N,G} box{128,128,1}; WGRAD x_c{K,M} box{128,128}
-  CUtensorMap tmSA;   // A scales: FWD/DGRAD k-group words {pitchM, Kc/128} box{132,1}; WGRAD dy_sc{N,S} box{128,4}
-  CUtensorMap tmSB;   // stacked B scales: FWD {pitchGN, K/128} box{224,1}; DGRAD Wsc{K,G*N32} box{224,4}; WGRAD x_sc{K,S} box{224,4}
+  CUtensorMap tmSA;   // A scale atoms (u32 {128, atoms, k-groups}) box{128,1,1}
+  CUtensorMap tmSB;   // stacked B scale atoms box{128,2,1}
   CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,32,1}
-  const int64_t* offsets;
+  const int64_t* offsets;      // this launch's G+1 offsets
+  const int64_t* offsets_all;  // every group's offsets (WGRAD scale k-groups of earlier groups)
   int32_t* status;
   int64_t out_rows;
   void* out;
   const __nv_bfloat16* bias;
   int G;
+  int g0;  // index of this launch's first group
   int N, K;
-  int n32;  // ceil(N/32): columnwise scale rows per weight group
   int has_bias;
   int accumulate;
 };
@@ -95,7 +104,7 @@ struct MxParams {
 template <bool PG>
 struct MxPG {
   CUtensorMap tm[kPG];   // FWD/DGRAD: B codes of group g; WGRAD: main_grad of group g
-  CUtensorMap tms[kPG];  // FWD/DGRAD: B scales of group g
+  CUtensorMap tms[kPG];  // FWD/DGRAD: B scale atoms of group g
   const __nv_bfloat16* bias[kPG];
   __device__ const CUtensorMap* map(int g) const { return &tm[g]; }
   __device__ const CUtensorMap* smap(int g) const { return &tms[g]; }
@@ -111,17 +120,24 @@ struct MxPG<false> {
 
 struct Tile {
   int g, num_kb, mt, nt;
-  int64_t r0, r1;
+  int64_t r0;   // FWD/DGRAD: first A row of the tile (a multiple of 128); WGRAD: group start
+  int64_t rlo;  // group start
+  int64_t r1;   // group end
 };
 
 __device__ __forceinline__ int cdiv(int64_t a, int b) { return static_cast<int>((a + b - 1) / b); }
 
+// First A row of a group's fprop / dgrad tiles: the group start rounded down
+// to the 128-row scale atoms.
+__device__ __forceinline__ int64_t atom_floor(int64_t r) { return r & ~int64_t(127); }
+
 template <int MODE, int CG>
-__device__ __forceinline__ int tiles_of_group(int64_t m, const MxParams& p) {
+__device__ __forceinline__ int tiles_of_group(int64_t o0, int64_t o1, const MxParams& p) {
   constexpr int TMt = CfgMX<MODE, CG>::kTileM;
-  if (MODE == kFwd) return m > 0 ? cdiv(m, TMt) * cdiv(p.N, TN) : 0;
-  if (MODE == kDgrad) return m > 0 ? cdiv(m, TMt) * cdiv(p.K, TN) : 0;
-  return (m > 0 || !p.accumulate) ? cdiv(p.N, TMt) * cdiv(p.K, TN) : 0;
+  const int64_t m = o1 > o0 ? o1 - o0 : 0;
+  if (MODE == kWgrad) return (m > 0 || !p.accumulate) ? cdiv(p.N, TMt) * cdiv(p.K, TN) : 0;
+  if (m == 0) return 0;
+  return cdiv(o1 - atom_floor(o0), TMt) * cdiv(MODE == kFwd ? p.N : p.K, TN);
 }
 
 template <int MODE, int CG>
@@ -137,7 +153,7 @@ __device__ __forceinline__ Tile decode(int t, const int* prefix, const MxParams&
   const int local = t - prefix[lo];
   const int64_t o0 = __ldg(p.offsets + lo), o1 = __ldg(p.offsets + lo + 1);
   const int64_t m = o1 > o0 ? o1 - o0 : 0;
-  const int mtg = (MODE == kWgrad) ? cdiv(p.N, TMt) : cdiv(m, TMt);
+  const int mtg = (MODE == kWgrad) ? cdiv(p.N, TMt) : cdiv(o0 + m - atom_floor(o0), TMt);
   const int ntg = cdiv(MODE == kFwd ? p.N : p.K, TN);
   const int band = local / (kBand * ntg);
   const int base_mt = band * kBand;
@@ -145,13 +161,13 @@ __device__ __forceinline__ Tile decode(int t, const int* prefix, const MxParams&
   const int within = local - band * kBand * ntg;
   tl.mt = base_mt + within % bh;
   tl.nt = within / bh;
+  tl.rlo = o0;
+  tl.r1 = o0 + m;
   if (MODE == kWgrad) {
     tl.r0 = o0;
-    tl.r1 = o0 + m;
     tl.num_kb = cdiv(m, BK);
   } else {
-    tl.r0 = o0 + static_cast<int64_t>(tl.mt) * TMt;
-    tl.r1 = o0 + m;
+    tl.r0 = atom_floor(o0) + static_cast<int64_t>(tl.mt) * TMt;
     tl.num_kb = (MODE == kFwd ? p.K : p.N) / BK;
   }
   return tl;
@@ -169,27 +185,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Word offset of row i inside the packed scale blocks (512 bytes per 128 rows).
-__device__ __forceinline__ int packed_word(int i) {
-  return (i >> 7) * 128 + (i & 31) * 4 + ((i >> 5) & 3);
-}
-
-// Repack one operand's raw scales of a stage into the tcgen05.cp layout.
-// Rowwise source: words (four scales of row i in word skip + i).  Columnwise
-// source: 4 rows of `pitch` bytes (scale of block kb of row i at kb*pitch + i).
-template <bool COLWISE>
-__device__ __forceinline__ void pack_scales(const uint8_t* raw, uint32_t* packed, int R, int pitch, int skip,
-                                            int lane) {
-  for (int i = lane; i < R; i += 32) {
-    uint32_t w;
-    if (COLWISE) {
-      w = static_cast<uint32_t>(raw[i]) | (static_cast<uint32_t>(raw[pitch + i]) << 8) |
-          (static_cast<uint32_t>(raw[2 * pitch + i]) << 16) | (static_cast<uint32_t>(raw[3 * pitch + i]) << 24);
-    } else {
-      w = reinterpret_cast<const uint32_t*>(raw)[skip + i];
-    }
-    packed[packed_word(i)] = w;
+// Ragged wgrad contraction: zero the code rows [valid, to) of this CTA's stage
+// (A: one 128-column chunk; B: kBChunks chunks; 128 bytes per contraction
+// row) -- the rows of the last partial 32-row MMA step that belong to the
+// next group.  Steps wholly past the group's end are skipped by the MMA.
+template <int MODE, int CG>
+__device__ __forceinline__ void zero_tail_rows(uint8_t* sa, uint8_t* sb, int valid, int to, int lane) {
+  constexpr int kChunks = 1 + CfgMX<MODE, CG>::kBChunks;
+  const int nrows = to - valid;
+  if (nrows <= 0) return;
+  const int per_chunk = nrows * 8;  // 16-byte pieces per chunk
+  for (int idx = lane; idx < kChunks * per_chunk; idx += 32) {
+    const int chunk = idx / per_chunk;
+    const int rem = idx - chunk * per_chunk;
+    const int r = valid + (rem >> 3);
+    uint8_t* base = chunk == 0 ? sa : (sb + (chunk - 1) * 16384);
+    *reinterpret_cast<uint4*>(base + r * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
   }
+  fence_proxy_async_smem();
 }
 
 template <int MODE, int CG, bool PG>
@@ -201,15 +214,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* empty = full + C::kStages;
-  uint64_t* ready = empty + C::kStages;  // stage's scales repacked (both CTAs of a pair)
-  uint64_t* tfull = ready + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* skip_flag = abort_flag + 1;
   int* prefix = reinterpret_cast<int*>(smem + C::kPrefixOffset);  // tiles before group g
-  int* bprefix = prefix + (p.G + 1);                             // 32-row blocks before group g
+  int* qprefix = prefix + (p.G + 1);                             // WGRAD: scale k-groups before group g
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -220,9 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     *skip_flag = (p.status != nullptr && *reinterpret_cast<volatile int32_t*>(p.status) != 0) ? 1 : 0;
     *abort_flag = 0;
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], (CG == 2 && leader) ? 2 : 1);  // leader: own TMA + peer's relay
       mbar_init(&empty[s], 1);
-      mbar_init(&ready[s], (CG == 2 && leader) ? 2 : 1);  // leader: both CTAs' repack warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -251,26 +262,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int npairs = (CG == 2) ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (warp == 0) {
-    int carry = 0, bcarry = 0;
+    // WGRAD: scale k-groups of the groups before this launch (per-group
+    // main_grad launches cover 64 groups each)
+    int qbase = 0;
+    if (MODE == kWgrad) {
+      for (int base = 0; base < p.g0; base += 32) {
+        const int i = base + lane;
+        int qc = 0;
+        if (i < p.g0) {
+          const int64_t m = __ldg(p.offsets_all + i + 1) - __ldg(p.offsets_all + i);
+          qc = m > 0 ? cdiv(m, 128) : 0;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) qc += __shfl_xor_sync(0xffffffffu, qc, off);
+        qbase += qc;
+      }
+    }
+    int carry = 0, qcarry = qbase;
     for (int base = 0; base < p.G; base += 32) {
       const int i = base + lane;
-      int cnt = 0, bc = 0;
+      int cnt = 0, qc = 0;
       if (i < p.G) {
-        const int64_t m = __ldg(p.offsets + i + 1) - __ldg(p.offsets + i);
-        cnt = tiles_of_group<MODE, CG>(m, p);
-        bc = m > 0 ? cdiv(m, 32) : 0;
+        const int64_t o0 = __ldg(p.offsets + i), o1 = __ldg(p.offsets + i + 1);
+        cnt = tiles_of_group<MODE, CG>(o0, o1, p);
+        qc = o1 > o0 ? cdiv(o1 - o0, 128) : 0;
       }
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, cnt, off);
-        const int u = __shfl_up_sync(0xffffffffu, bc, off);
-        if (lane >= off) { cnt += v; bc += u; }
+        const int u = __shfl_up_sync(0xffffffffu, qc, off);
+        if (lane >= off) { cnt += v; qc += u; }
       }
-      if (i < p.G) { prefix[i + 1] = carry + cnt; bprefix[i + 1] = bcarry + bc; }
+      if (i < p.G) { prefix[i + 1] = carry + cnt; qprefix[i + 1] = qcarry + qc; }
       carry += __shfl_sync(0xffffffffu, cnt, 31);
-      bcarry += __shfl_sync(0xffffffffu, bc, 31);
+      qcarry += __shfl_sync(0xffffffffu, qc, 31);
     }
-    if (lane == 0) { prefix[0] = 0; bprefix[0] = 0; }
+    if (lane == 0) { prefix[0] = 0; qprefix[0] = qbase; }
   } else if (warp == 1) {
     if (CG == 2) {
       tmem_alloc_pair(tmem_slot, 512);
@@ -296,44 +323,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int t = pair; t < total && !*abort_flag; t += npairs) {
         const Tile tl = decode<MODE, CG>(t, prefix, p);
+        const int n0 = tl.nt * TN;  // first B operand row of the tile
         for (int kb = 0; kb < tl.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { report_abort(abort_flag, p.status); break; }
-          uint8_t* sa = smem + stage * C::kOpStage;
+          uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
-          uint8_t* sf = smem + C::kSfOffset + stage * kSfStage;
+          uint8_t* sf = sb + C::kBAlloc;
           uint64_t* bar = &full[stage];
           mbar_arrive_expect_tx(bar, C::kTx);
-          const int n0 = tl.nt * TN;  // first B row (all 224 for the scales)
-          const int32_t ra = static_cast<int32_t>(tl.r0 + hr);
-          if (MODE == kFwd) {
+          if (MODE == kFwd || MODE == kDgrad) {
+            const int32_t ra = static_cast<int32_t>(tl.r0 + hr);  // multiple of 128
             tma_load_2d(sa, &p.tmA, bar, kb * BK, ra);
-            tma_load_2d(sf, &p.tmSA, bar, ra & ~3, kb);
+            tma_load_3d(sf, &p.tmSA, bar, 0, ra >> 7, kb);
+          }
+          if (MODE == kFwd) {
             if (PG) {
               tma_load_2d(sb, pg.map(tl.g), bar, kb * BK, n0 + hb);
-              tma_load_2d(sf + kRawB, pg.smap(tl.g), bar, n0, kb);
+              tma_load_3d(sf + kSfABytes, pg.smap(tl.g), bar, 0, n0 >> 7, kb);
             } else {
               tma_load_3d(sb, &p.tmB, bar, kb * BK, n0 + hb, tl.g);
-              tma_load_2d(sf + kRawB, &p.tmSB, bar, tl.g * p.N + n0, kb);
+              tma_load_3d(sf + kSfABytes, &p.tmSB, bar, 0, tl.g * (p.N >> 7) + (n0 >> 7), kb);
             }
           } else if (MODE == kDgrad) {
-            tma_load_2d(sa, &p.tmA, bar, kb * BK, ra);
-            tma_load_2d(sf, &p.tmSA, bar, ra & ~3, kb);
 #pragma unroll
-            for (int c = 0; c < (CG == 1 ? 2 : 1); ++c) {
+            for (int c = 0; c < C::kBChunks; ++c) {
               if (PG) tma_load_2d(sb + c * 16384, pg.map(tl.g), bar, n0 + hb + c * 128, kb * BK);
               else    tma_load_3d(sb + c * 16384, &p.tmB, bar, n0 + hb + c * 128, kb * BK, tl.g);
             }
-            if (PG) tma_load_2d(sf + kRawB, pg.smap(tl.g), bar, n0, 4 * kb);
-            else    tma_load_2d(sf + kRawB, &p.tmSB, bar, n0, tl.g * p.n32 + 4 * kb);
+            if (PG) tma_load_3d(sf + kSfABytes, pg.smap(tl.g), bar, 0, n0 >> 7, kb);
+            else    tma_load_3d(sf + kSfABytes, &p.tmSB, bar, 0, n0 >> 7, tl.g * (p.N >> 7) + kb);
           } else {
             const int32_t row = static_cast<int32_t>(tl.r0 + kb * BK);
-            const int32_t brow = bprefix[tl.g] + 4 * kb;  // scale row of this stage's first block
+            const int kq = qprefix[tl.g] + kb;  // scale k-group of this stage
             const int m0 = tl.mt * TMt + hr;
             tma_load_2d(sa, &p.tmA, bar, m0, row);
 #pragma unroll
-            for (int c = 0; c < (CG == 1 ? 2 : 1); ++c) tma_load_2d(sb + c * 16384, &p.tmB, bar, n0 + hb + c * 128, row);
-            tma_load_2d(sf, &p.tmSA, bar, m0, brow);
-            tma_load_2d(sf + kRawB, &p.tmSB, bar, n0, brow);
+            for (int c = 0; c < C::kBChunks; ++c) tma_load_2d(sb + c * 16384, &p.tmB, bar, n0 + hb + c * 128, row);
+            tma_load_3d(sf, &p.tmSA, bar, 0, m0 >> 7, kq);
+            tma_load_3d(sf + kSfABytes, &p.tmSB, bar, 0, n0 >> 7, kq);
           }
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -353,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
+      uint32_t kiter = 0;
       for (int t = pair; t < total; t += npairs, ++it) {
         const Tile tl = decode<MODE, CG>(t, prefix, p);
         const int buf = it & 1;
@@ -363,38 +391,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * TN;
+        // the tile's first B row sits 32 * sh rows into the first loaded atom
+        const uint32_t sh = static_cast<uint32_t>((tl.nt * TN) & 127) >> 5;
         bool ok = true;
-        for (int kb = 0; kb < tl.num_kb; ++kb) {
-          // stage landed and repacked in this CTA (and, for a pair, in the peer)
-          const bool rdy = mbar_wait(&full[stage], phase, abort_flag) &&
-                           (CG == 2 ? mbar_wait_acq_cluster(&ready[stage], phase, abort_flag)
-                                    : mbar_wait(&ready[stage], phase, abort_flag));
-          if (!__all_sync(0xffffffffu, rdy)) {
+        for (int kb = 0; kb < tl.num_kb; ++kb, ++kiter) {
+          int ksteps = BK / 32;
+          int valid = BK;
+          if (MODE == kWgrad && kb == tl.num_kb - 1) {
+            valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
+            if (valid < BK) ksteps = (valid + 31) >> 5;
+          }
+          // the peer zeroed rows of its stage before relaying: acquire at
+          // cluster scope so those writes are visible to the pair's MMAs
+          const bool peer_zeroed = CG == 2 && MODE == kWgrad && valid < BK;
+          const bool landed = peer_zeroed ? mbar_wait_acq_cluster(&full[stage], phase, abort_flag)
+                                          : mbar_wait(&full[stage], phase, abort_flag);
+          if (!__all_sync(0xffffffffu, landed)) {
             report_abort(abort_flag, p.status);
             ok = false;
             break;
           }
           tc_fence_after();
-          uint8_t* sa = smem + stage * C::kOpStage;
+          uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
-          uint8_t* sf = smem + C::kSfOffset + stage * kSfStage;
-          int ksteps = BK / 32;
-          if (MODE == kWgrad && kb == tl.num_kb - 1) {
-            const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
-            if (valid < BK) ksteps = (valid + 31) >> 5;
-          }
+          uint8_t* sf = sb + C::kBAlloc;
+          if (MODE == kWgrad && valid < BK) zero_tail_rows<MODE, CG>(sa, sb, valid, ksteps * 32, lane);
+          __syncwarp();
           if (lane == 0) {
-            const uint32_t sfa = tmem_base + kSfCol0 + stage * C::kSfSlot, sfb = sfa + 4;
-            const uint32_t pa = smem_u32(sf + kPackA), pb = smem_u32(sf + kPackB);
+            const uint32_t sfa = tmem_base + kSfCol0 + (kiter & (kSfSlots - 1)) * kSfSlotCols;
+            const uint32_t sfb0 = sfa + 4;
+            const uint32_t pa = smem_u32(sf), pb = smem_u32(sf + kSfABytes);
             if (CG == 2) {
               tmem_cp_32x128b_x4_pair(sfa, smem_desc_sf(pa));
-              tmem_cp_32x128b_x4_pair(sfb, smem_desc_sf(pb));
-              tmem_cp_32x128b_x4_pair(sfb + 4, smem_desc_sf(pb + 512));
+#pragma unroll
+              for (int a = 0; a < kAtomsB; ++a) tmem_cp_32x128b_x4_pair(sfb0 + 4 * a, smem_desc_sf(pb + 512 * a));
             } else {
               tmem_cp_32x128b_x4(sfa, smem_desc_sf(pa));
-              tmem_cp_32x128b_x4(sfb, smem_desc_sf(pb));
-              tmem_cp_32x128b_x4(sfb + 4, smem_desc_sf(pb + 512));
+#pragma unroll
+              for (int a = 0; a < kAtomsB; ++a) tmem_cp_32x128b_x4(sfb0 + 4 * a, smem_desc_sf(pb + 512 * a));
             }
+            const uint32_t sfb = sfb0 + sh;
             const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
             for (int ks = 0; ks < ksteps; ++ks) {
               const uint64_t ad = C::kAMN ? smem_desc_sw128(a0 + ks * 4096, 16384, 1024)
@@ -430,55 +466,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_bounded(mma_done, 0);
       }
       __syncwarp();
-    }
-  } else if (warp == 6) {
-    // ===================== scale repack (and wgrad tail zeroing) =====================
-    int stage = 0;
-    uint32_t phase = 0;
-    const uint32_t ready_leader = (CG == 2) ? mapa_shared(smem_u32(ready), 0) : 0u;
-    for (int t = pair; t < total; t += npairs) {
-      const Tile tl = decode<MODE, CG>(t, prefix, p);
-      bool ok = true;
-      for (int kb = 0; kb < tl.num_kb; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
-          report_abort(abort_flag, p.status);
-          ok = false;
-          break;
-        }
-        uint8_t* sa = smem + stage * C::kOpStage;
-        uint8_t* sb = sa + C::kABytes;
-        uint8_t* sf = smem + C::kSfOffset + stage * kSfStage;
-        if (MODE == kWgrad && kb == tl.num_kb - 1) {
-          // ragged contraction: zero the code rows of the last partial 32-row
-          // MMA step (A: one 128-column chunk, B: 1 or 2; 128 bytes per row);
-          // the MMA warp skips the steps past the group's end
-          const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
-          if (valid < BK) {
-            constexpr int kChunks = 1 + (CG == 1 ? 2 : 1);
-            const int nrows = ((valid + 31) >> 5) * 32 - valid;
-            const int per_chunk = nrows * 8;
-            for (int idx = lane; idx < kChunks * per_chunk; idx += 32) {
-              const int chunk = idx / per_chunk;
-              const int rem = idx - chunk * per_chunk;
-              const int r = valid + (rem >> 3);
-              uint8_t* base = chunk == 0 ? sa : (sb + (chunk - 1) * 16384);
-              *reinterpret_cast<uint4*>(base + r * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+    } else {
+      // ===================== peer: stage relay =====================
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = pair; t < total; t += npairs) {
+        const Tile tl = decode<MODE, CG>(t, prefix, p);
+        bool ok = true;
+        for (int kb = 0; kb < tl.num_kb; ++kb) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+            report_abort(abort_flag, p.status);
+            ok = false;
+            break;
+          }
+          bool zeroed = false;
+          if (MODE == kWgrad && kb == tl.num_kb - 1) {
+            const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
+            if (valid < BK) {
+              uint8_t* sa = smem + stage * C::kStageBytes;
+              zero_tail_rows<MODE, CG>(sa, sa + C::kABytes, valid, ((valid + 31) >> 5) * 32, lane);
+              zeroed = true;
             }
           }
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
+            if (zeroed) mbar_arrive_cluster_release(leader_full);  // the leader's MMA reads our zeroes
+            else        mbar_arrive_cluster(leader_full);
+          }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
-        pack_scales<C::kSfaCol != 0>(sf, reinterpret_cast<uint32_t*>(sf + kPackA), 128, 128,
-                                     static_cast<int>((tl.r0 + hr) & 3), lane);
-        pack_scales<C::kSfbCol != 0>(sf + kRawB, reinterpret_cast<uint32_t*>(sf + kPackB), TN, TN, 0, lane);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          // the leader's MMAs read this CTA's zeroed codes and packed scales
-          if (CG == 2) mbar_arrive_cluster_release(ready_leader + stage * 8);
-          else         mbar_arrive(&ready[stage]);
-        }
-        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        if (!ok) break;
       }
-      if (!ok) break;
     }
   } else {
     // ===================== epilogue (warps 2..5, both CTAs) =====================
@@ -507,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (MODE != kWgrad) {
         const int Nout = (MODE == kFwd) ? p.N : p.K;
         const int64_t row = tl.r0 + hr + row_in_tile;
-        const bool row_ok = row >= 0 && row < tl.r1 && row < p.out_rows;
+        const bool row_ok = row >= tl.rlo && row < tl.r1 && row < p.out_rows;
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
         const __nv_bfloat16* bias = nullptr;
         if (MODE == kFwd && p.has_bias) bias = PG ? pg.b(tl.g) : (p.bias + static_cast<int64_t>(tl.g) * p.N);
@@ -619,6 +638,17 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64
   return encode_tmap(m, dt, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Scale atoms as a u32 tensor {128 words, atoms, k-groups}: `atoms` 512-byte
+// atoms per k-group, consecutive k-groups `kstride` atoms apart; the box is
+// `box_atoms` consecutive atoms of one k-group.
+bool map_atoms(CUtensorMap* m, const void* base, uint64_t atoms, uint64_t kgroups, uint64_t kstride,
+               uint32_t box_atoms) {
+  const uint64_t dims[3] = {128, atoms, kgroups};
+  const uint64_t strides[2] = {512, kstride * 512};
+  const uint32_t box[3] = {128, box_atoms, 1};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 template <int MODE, int CG>
 constexpr int mx_smem_bytes(int G) {
   return CfgMX<MODE, CG>::kPrefixOffset + 2 * (G + 1) * 4 + 1024;
@@ -685,9 +715,7 @@ template <int MODE, int CG>
 gl_status mx_mode(const MxCall& c) {
   using Cf = CfgMX<MODE, CG>;
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  const auto U32 = CU_TENSOR_MAP_DATA_TYPE_UINT32;
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
-  const auto NOSW = CU_TENSOR_MAP_SWIZZLE_NONE;
   MxParams prm;
   memset(&prm, 0, sizeof(prm));
   prm.status = c.status;
@@ -695,25 +723,27 @@ gl_status mx_mode(const MxCall& c) {
   prm.out = c.out;
   prm.N = c.N;
   prm.K = c.K;
-  prm.n32 = (c.N + 31) / 32;
   prm.accumulate = c.accumulate;
   prm.has_bias = (MODE == kFwd && c.bias != nullptr) ? 1 : 0;
+  prm.offsets_all = c.offsets;
   const uint64_t M = c.M > 0 ? static_cast<uint64_t>(c.M) : 1;
-  const uint64_t pitchM = (M + 3) / 4 * 4;
-  const uint64_t S = (M + 31) / 32 + c.G;  // columnwise scale rows allocated by the caller
+  const uint64_t RB = (M + 127) / 128;                  // row atoms of x / dy rowwise scales
+  const uint64_t KQ = RB + static_cast<uint64_t>(c.G);  // bound on x_c / dy_c scale k-groups
+  const uint64_t NA = c.N / 128, KA = c.K / 128;        // 128-row atoms along N and K
+  const uint64_t G = static_cast<uint64_t>(c.G);
   const uint32_t BR = Cf::kBRows;
   bool ok = true;
   if (MODE == kFwd) {
     ok &= map2(&prm.tmA, c.a, c.K, M, c.K, 128, 128, U8, SW);
-    ok &= map2(&prm.tmSA, c.sa, pitchM, c.K / 128, pitchM * 4, 128 + 4, 1, U32, NOSW);
+    ok &= map_atoms(&prm.tmSA, c.sa, RB, KA, RB, 1);
   } else if (MODE == kDgrad) {
     ok &= map2(&prm.tmA, c.a, c.N, M, c.N, 128, 128, U8, SW);
-    ok &= map2(&prm.tmSA, c.sa, pitchM, c.N / 128, pitchM * 4, 128 + 4, 1, U32, NOSW);
+    ok &= map_atoms(&prm.tmSA, c.sa, RB, NA, RB, 1);
   } else {
     ok &= map2(&prm.tmA, c.a, c.N, M, c.N, 128, 128, U8, SW);
     ok &= map2(&prm.tmB, c.b, c.K, M, c.K, 128, 128, U8, SW);
-    ok &= map2(&prm.tmSA, c.sa, c.N, S, c.N, 128, 4, U8, NOSW);
-    ok &= map2(&prm.tmSB, c.sb, c.K, S, c.K, TN, 4, U8, NOSW);
+    ok &= map_atoms(&prm.tmSA, c.sa, NA, KQ, NA, 1);
+    ok &= map_atoms(&prm.tmSB, c.sb, KA, KQ, KA, kAtomsB);
   }
   if (!ok) return GL_ERR_UNSUPPORTED;
 
@@ -722,18 +752,18 @@ gl_status mx_mode(const MxCall& c) {
   const bool bias_ok = !prm.has_bias || c.bias->mode == GL_STACKED;
   if (stacked && bias_ok) {
     if (MODE == kFwd) {
-      const uint64_t GN = static_cast<uint64_t>(c.G) * c.N, pitchGN = (GN + 3) / 4 * 4;
       ok &= map3(&prm.tmB, c.w.base, c.K, c.N, c.G, 1, 128, BR, U8);
-      ok &= map2(&prm.tmSB, c.ws.base, pitchGN, c.K / 128, pitchGN * 4, TN, 1, U32, NOSW);
+      ok &= map_atoms(&prm.tmSB, c.ws.base, G * NA, KA, G * NA, kAtomsB);  // rows G*N, cols K
     } else if (MODE == kDgrad) {
       ok &= map3(&prm.tmB, c.w.base, c.K, c.N, c.G, 1, 128, 128, U8);
-      ok &= map2(&prm.tmSB, c.ws.base, c.K, static_cast<uint64_t>(c.G) * prm.n32, c.K, TN, 4, U8, NOSW);
+      ok &= map_atoms(&prm.tmSB, c.ws.base, KA, G * NA, KA, kAtomsB);  // G groups of N/128 k-groups
     } else {
       ok &= map3(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
     }
     if (!ok) return GL_ERR_UNSUPPORTED;
     prm.offsets = c.offsets;
     prm.G = c.G;
+    prm.g0 = 0;
     if (prm.has_bias) prm.bias = reinterpret_cast<const __nv_bfloat16*>(c.bias->base);
     MxPG<false> none{0};
     return mx_launch<MODE, CG, false>(prm, none, c.G, c.stream);
@@ -753,20 +783,18 @@ gl_status mx_mode(const MxCall& c) {
       }
       const void* wp = group_ptr(c.w, g, static_cast<size_t>(c.N) * c.K);
       if (MODE == kFwd) {
-        const uint64_t pitchN = (static_cast<uint64_t>(c.N) + 3) / 4 * 4;
-        const uint64_t GN = static_cast<uint64_t>(c.G) * c.N, pitchGN = (GN + 3) / 4 * 4;
         ok &= map2(&pga->tm[i], wp, c.K, c.N, c.K, 128, BR, U8, SW);
         if (c.ws.mode == GL_STACKED) {
-          // group g's rows of the stacked [K/128][pitch(G*N)] scale array
-          const void* sp = static_cast<const uint8_t*>(c.ws.base) + static_cast<size_t>(g) * c.N * 4;
-          ok &= map2(&pga->tms[i], sp, c.N, c.K / 128, pitchGN * 4, TN, 1, U32, NOSW);
+          // group g's N/128 atoms inside each k-group of the stacked [G*N, K] atoms
+          const void* sp = static_cast<const uint8_t*>(c.ws.base) + static_cast<size_t>(g) * NA * 512;
+          ok &= map_atoms(&pga->tms[i], sp, NA, KA, G * NA, kAtomsB);
         } else {
-          ok &= map2(&pga->tms[i], c.ws.ptrs[g], pitchN, c.K / 128, pitchN * 4, TN, 1, U32, NOSW);
+          ok &= map_atoms(&pga->tms[i], c.ws.ptrs[g], NA, KA, NA, kAtomsB);
         }
       } else {
         ok &= map2(&pga->tm[i], wp, c.K, c.N, c.K, 128, 128, U8, SW);
-        const void* sp = group_ptr(c.ws, g, static_cast<size_t>(prm.n32) * c.K);
-        ok &= map2(&pga->tms[i], sp, c.K, prm.n32, c.K, TN, 4, U8, NOSW);
+        const void* sp = group_ptr(c.ws, g, static_cast<size_t>(NA) * KA * 512);
+        ok &= map_atoms(&pga->tms[i], sp, KA, NA, KA, kAtomsB);
       }
       if (prm.has_bias)
         pga->bias[i] = reinterpret_cast<const __nv_bfloat16*>(group_ptr(*c.bias, g, static_cast<size_t>(c.N) * 2));
@@ -774,6 +802,7 @@ gl_status mx_mode(const MxCall& c) {
     if (!ok) { st = GL_ERR_UNSUPPORTED; break; }
     prm.offsets = c.offsets + g0;
     prm.G = cg;
+    prm.g0 = g0;
     st = mx_launch<MODE, CG, true>(prm, *pga, cg, c.stream);
   }
   delete pga;

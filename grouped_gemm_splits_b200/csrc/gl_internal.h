@@ -49,11 +49,11 @@ gl_status launch_grouped_gemm(const GemmCall& c);
 struct MxCall {
   int mode;
   const void* a;           // A codes: FWD x, DGRAD dy (rowwise); WGRAD dy (columnwise)
-  const void* sa;          // A scales: k-group rowwise (FWD/DGRAD) or columnwise [S, N] (WGRAD)
+  const void* sa;          // A scale atoms: rowwise (FWD/DGRAD) or columnwise (WGRAD), GL_SCALES_MMA
   const void* b;           // WGRAD: x columnwise codes
-  const void* sb;          // WGRAD: x columnwise scales [S, K]
+  const void* sb;          // WGRAD: x columnwise scale atoms
   gl_grouped w;            // FWD: W rowwise codes; DGRAD: W columnwise codes
-  gl_grouped ws;           // FWD: W k-group rowwise scales; DGRAD: W columnwise scales
+  gl_grouped ws;           // FWD: W rowwise scale atoms; DGRAD: W columnwise scale atoms
   const gl_grouped* bias;  // FWD (nullable)
   gl_grouped out_grouped;  // WGRAD main_grad
   void* out;
@@ -64,7 +64,7 @@ struct MxCall {
   int64_t M;
   int N, K;
   int accumulate;
-  int cta_pair;  // 1: 256x224 tiles on CTA pairs; 0: 128x224 tiles per CTA
+  int cta_pair;  // 1: 256x192 tiles on CTA pairs; 0: 128x192 tiles per CTA
   cudaStream_t stream;
 };
 

@@ -57,9 +57,11 @@ __global__ void __launch_bounds__(kQThreads, 4)
     quantize_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int cols,
                     const int64_t* __restrict__ row_offsets, int G, const int32_t* __restrict__ status,
                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r,
-                    uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, int kgroup_pitch) {
+                    uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, int64_t scales_c_bytes,
+                    int mma_layout) {
   extern __shared__ int64_t qsmem[];
-  int64_t* bprefix = qsmem;  // G+1: first block index of each group (ragged mode)
+  int64_t* bprefix = qsmem;        // G+1: first 32-row block of each group (ragged mode)
+  int64_t* qprefix = qsmem + G + 1;  // G+1: first 128-row k-group of each group (ragged mode)
   __shared__ float cmax[kQThreads / 32][kQCols];
   __shared__ float csf[kQCols];
   if (status != nullptr && *status != 0) return;
@@ -67,26 +69,32 @@ __global__ void __launch_bounds__(kQThreads, 4)
 
   const int64_t per = (row_offsets == nullptr) ? rows / G : 0;
   const int64_t bpg = (per + kQRows - 1) / kQRows;  // blocks per group (uniform mode)
+  const int64_t qpg = (per + 127) / 128;            // k-groups per group (uniform mode)
+  const int64_t mma_rb = (rows + 127) / 128;        // 128-row blocks (rowwise MMA layout)
+  const int mma_cb = cols / 128;                    // 128-column blocks (columnwise MMA layout)
   int64_t nblocks;
   if (row_offsets != nullptr) {
     if (warp == 0) {
-      int64_t carry = 0;
+      int64_t carry = 0, qcarry = 0;
       for (int base = 0; base < G; base += 32) {
         const int i = base + lane;
-        int64_t cnt = 0;
+        int64_t cnt = 0, qc = 0;
         if (i < G) {
           const int64_t m = row_offsets[i + 1] - row_offsets[i];
           cnt = m > 0 ? (m + kQRows - 1) / kQRows : 0;
+          qc = m > 0 ? (m + 127) / 128 : 0;
         }
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
           const int64_t u = __shfl_up_sync(0xffffffffu, cnt, off);
-          if (lane >= off) cnt += u;
+          const int64_t w = __shfl_up_sync(0xffffffffu, qc, off);
+          if (lane >= off) { cnt += u; qc += w; }
         }
-        if (i < G) bprefix[i + 1] = carry + cnt;
+        if (i < G) { bprefix[i + 1] = carry + cnt; qprefix[i + 1] = qcarry + qc; }
         carry += __shfl_sync(0xffffffffu, cnt, 31);
+        qcarry += __shfl_sync(0xffffffffu, qc, 31);
       }
-      if (lane == 0) bprefix[0] = 0;
+      if (lane == 0) { bprefix[0] = 0; qprefix[0] = 0; }
     }
     __syncthreads();
     nblocks = bprefix[G];
@@ -181,12 +189,13 @@ __global__ void __launch_bounds__(kQThreads, 4)
           q.y = e4m3x4(v[i][4] * s, v[i][5] * s, v[i][6] * s, v[i][7] * s);
           *reinterpret_cast<uint2*>(codes_r + row * cols + col) = q;
           if ((c8 & 3) == 0) {
-            // row-major [rows, cols/32], or k-group-major words: the four
-            // scales of k-blocks 4j..4j+3 of a row form word (j, row) of a
-            // [cols/128][kgroup_pitch] array (what the MXFP8 GEMM loads per stage)
+            // row-major [rows, cols/32], or the tcgen05 scale-factor atoms:
+            // 512 bytes per (k-group of 4 blocks, 128 rows), row i of the
+            // atom at byte (i%32)*16 + ((i/32)%4)*4 + block
             const int64_t kb = col / 32;
-            const int64_t at = kgroup_pitch > 0 ? ((kb >> 2) * kgroup_pitch + row) * 4 + (kb & 3)
-                                                : row * (cols / 32) + kb;
+            const int64_t at = mma_layout ? ((kb >> 2) * mma_rb + (row >> 7)) * 512 + (row & 31) * 16 +
+                                                ((row >> 5) & 3) * 4 + (kb & 3)
+                                          : row * (cols / 32) + kb;
             scales_r[at] = static_cast<uint8_t>(e + 127);
           }
         }
@@ -209,9 +218,18 @@ __global__ void __launch_bounds__(kQThreads, 4)
         const int e = mx_scale_exp(a);
         csf[tid] = pow2_neg(e);
         const int ccol = cc * kQCols + tid;
-        if (ccol < cols) {
-          const int64_t srow = (row_offsets != nullptr ? bprefix[g] : static_cast<int64_t>(g) * bpg) + j;
-          scales_c[srow * cols + ccol] = static_cast<uint8_t>(e + 127);
+        if (ccol < cols && vrows > 0) {
+          int64_t at;
+          if (mma_layout) {
+            // atom (k-group of the group's blocks 4t..4t+3, 128 columns)
+            const int64_t kq = (row_offsets != nullptr ? qprefix[g] : static_cast<int64_t>(g) * qpg) + (j >> 2);
+            at = (kq * mma_cb + (ccol >> 7)) * 512 + (ccol & 31) * 16 + ((ccol >> 5) & 3) * 4 + (j & 3);
+          } else {
+            at = ((row_offsets != nullptr ? bprefix[g] : static_cast<int64_t>(g) * bpg) + j) * cols + ccol;
+          }
+          // offsets that overlap (only possible without a status word) must
+          // not push a write past the documented allocation
+          if (at < scales_c_bytes) scales_c[at] = static_cast<uint8_t>(e + 127);
         }
       }
       __syncthreads();
@@ -245,13 +263,15 @@ __global__ void __launch_bounds__(kQThreads, 4)
 gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                           int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                           uint8_t* codes_c, uint8_t* scales_c, int scale_layout, cudaStream_t stream) {
-  const int smem = row_offsets != nullptr ? (G + 1) * static_cast<int>(sizeof(int64_t)) : 0;
+  const int smem = row_offsets != nullptr ? 2 * (G + 1) * static_cast<int>(sizeof(int64_t)) : 0;
   if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel), smem + 16 * 1024) != cudaSuccess)
     return GL_ERR_CUDA;
   const int grid = num_sms() * 4;
   quantize_kernel<<<grid, kQThreads, smem, stream>>>(
       static_cast<const __nv_bfloat16*>(src), rows, cols, row_offsets, G, status, codes_r,
-      scales_r, codes_c, scales_c, scale_layout == GL_SCALES_KGROUP ? static_cast<int>((rows + 3) / 4 * 4) : 0);
+      scales_r, codes_c, scales_c,
+      static_cast<int64_t>(gl_mxfp8_scale_bytes(rows, cols, G, 1, scale_layout)),
+      scale_layout == GL_SCALES_MMA ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
 }
 

@@ -21,10 +21,10 @@ _lib = None
 GL_OK, GL_ERR_INVALID, GL_ERR_UNSUPPORTED, GL_ERR_CUDA = 0, 1, 2, 3
 GL_DEV_NEG_SPLIT, GL_DEV_SUM_MISMATCH, GL_DEV_OUT_OVERFLOW, GL_DEV_TIMEOUT = 1, 2, 4, 8
 GL_STACKED, GL_PER_GROUP = 0, 1
-GL_SCALES_ROWMAJOR, GL_SCALES_KGROUP = 0, 1
+GL_SCALES_ROWMAJOR, GL_SCALES_MMA = 0, 1
 
 EXPORTED = ("gl_version", "gl_status_string", "gl_set_cta_pair", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
-            "group_quantize_mxfp8", "gl_fwd_mxfp8", "gl_dgrad_mxfp8", "gl_wgrad_mxfp8")
+            "group_quantize_mxfp8", "gl_mxfp8_scale_bytes", "gl_fwd_mxfp8", "gl_dgrad_mxfp8", "gl_wgrad_mxfp8")
 
 
 class GlGrouped(ctypes.Structure):
@@ -64,6 +64,8 @@ def load() -> ctypes.CDLL:
     L.gl_wgrad.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, vp]
     L.group_quantize_mxfp8.restype = i32
     L.group_quantize_mxfp8.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, vp, vp, i32, vp]
+    L.gl_mxfp8_scale_bytes.restype = ctypes.c_size_t
+    L.gl_mxfp8_scale_bytes.argtypes = [i64, i32, i32, i32, i32]
     L.gl_fwd_mxfp8.restype = i32
     L.gl_fwd_mxfp8.argtypes = [vp, vp, GlGrouped, GlGrouped, ctypes.POINTER(GlGrouped), vp, vp, i32, i64, i32,
                                i32, vp, i64, vp]
@@ -111,7 +113,7 @@ def _shape_nk(w: TensorOrList):
 GL_PAIRS_BF16, GL_PAIRS_MXFP8 = 1, 2
 
 
-def gl_set_cta_pair(bf16: bool = True, mxfp8: bool = False) -> None:
+def gl_set_cta_pair(bf16: bool = True, mxfp8: bool = True) -> None:
     """Tile shape of later GEMM launches: CTA pairs (256-row tiles) or single
     CTAs (128-row tiles), separately for the bf16 and the MXFP8 GEMMs."""
     _check(load().gl_set_cta_pair((GL_PAIRS_BF16 if bf16 else 0) | (GL_PAIRS_MXFP8 if mxfp8 else 0)),
@@ -184,26 +186,25 @@ def gl_wgrad(x: torch.Tensor, dy: torch.Tensor, offsets: torch.Tensor, status: t
     return main_grad
 
 
-def colwise_scale_rows_bound(rows: int, G: int) -> int:
-    """Rows to allocate for columnwise scales: ceil(rows/32) + G."""
-    return (rows + 31) // 32 + G
-
-
-def kgroup_pitch(rows: int) -> int:
-    """Row pitch (in 4-byte words) of k-group-major rowwise scales."""
-    return (rows + 3) // 4 * 4
+def mxfp8_scale_bytes(rows: int, cols: int, G: int, colwise: bool, mma: bool) -> int:
+    """Bytes to allocate for a scale array (``gl_mxfp8_scale_bytes``)."""
+    n = load().gl_mxfp8_scale_bytes(rows, cols, G, 1 if colwise else 0, GL_SCALES_MMA if mma else GL_SCALES_ROWMAJOR)
+    if n == 0:
+        raise GlError(f"gl_mxfp8_scale_bytes: invalid arguments ({rows}, {cols}, {G})")
+    return n
 
 
 def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] = None, G: int = 1,
                          rowwise: bool = True, colwise: bool = False,
                          status: Optional[torch.Tensor] = None, out: Optional[dict] = None,
-                         kgroup_scales: bool = False) -> dict:
+                         mma_scales: bool = False) -> dict:
     """MXFP8 cast of a bf16 [rows, cols] tensor (rows in G groups).
 
     Returns a dict with ``codes_r``/``scales_r`` (blocks along each row) and/or
-    ``codes_c``/``scales_c`` (blocks of 32 rows inside each group).  With
-    ``kgroup_scales`` the rowwise scales are a [cols/128, pitch, 4] array (the
-    form the MXFP8 GEMMs read) instead of [rows, cols/32].
+    ``codes_c``/``scales_c`` (blocks of 32 rows inside each group).  Scales are
+    [rows, cols/32] and [ceil(rows/32) + G, cols] arrays, or with
+    ``mma_scales`` flat byte arrays in the tcgen05 scale-factor layout that the
+    MXFP8 GEMMs read (``GL_SCALES_MMA``).
     """
     if src.dim() == 3:
         G = src.shape[0]
@@ -217,20 +218,23 @@ def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] 
     out = {} if out is None else out
     if rowwise:
         out.setdefault("codes_r", torch.empty(rows, cols, dtype=torch.uint8, device=dev))
-        if kgroup_scales:
-            out.setdefault("scales_r", torch.empty(cols // 128, kgroup_pitch(rows), 4, dtype=torch.uint8,
-                                                   device=dev))
+        if mma_scales:
+            out.setdefault("scales_r", torch.empty(mxfp8_scale_bytes(rows, cols, G, False, True),
+                                                   dtype=torch.uint8, device=dev))
         else:
             out.setdefault("scales_r", torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev))
     if colwise:
         out.setdefault("codes_c", torch.empty(rows, cols, dtype=torch.uint8, device=dev))
-        out.setdefault("scales_c", torch.empty(colwise_scale_rows_bound(rows, G), cols,
-                                               dtype=torch.uint8, device=dev))
+        if mma_scales:
+            out.setdefault("scales_c", torch.empty(mxfp8_scale_bytes(rows, cols, G, True, True),
+                                                   dtype=torch.uint8, device=dev))
+        else:
+            out.setdefault("scales_c", torch.empty((rows + 31) // 32 + G, cols, dtype=torch.uint8, device=dev))
     _check(load().group_quantize_mxfp8(
         src2.data_ptr(), rows, cols, _ptr(row_offsets), G, _ptr(status),
         _ptr(out.get("codes_r")) if rowwise else None, _ptr(out.get("scales_r")) if rowwise else None,
         _ptr(out.get("codes_c")) if colwise else None, _ptr(out.get("scales_c")) if colwise else None,
-        GL_SCALES_KGROUP if kgroup_scales else GL_SCALES_ROWMAJOR, _stream()), "group_quantize_mxfp8")
+        GL_SCALES_MMA if mma_scales else GL_SCALES_ROWMAJOR, _stream()), "group_quantize_mxfp8")
     return out
 
 
@@ -249,8 +253,8 @@ def _grouped_any(t: TensorOrList, G: int):
 def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorOrList, w_scales: TensorOrList,
                  bias: Optional[TensorOrList], offsets: torch.Tensor, status: torch.Tensor,
                  y: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """fprop on MXFP8 operands: x rowwise codes [M,K] + k-group scales; W rowwise
-    codes [G,N,K] (or G x [N,K]) + k-group scales."""
+    """fprop on MXFP8 operands: x rowwise codes [M,K] + scale atoms; W rowwise
+    codes [G,N,K] (or G x [N,K]) + scale atoms (all scales ``mma_scales``)."""
     G = offsets.numel() - 1
     M, K = x_codes.shape
     N = (w_codes if isinstance(w_codes, torch.Tensor) else w_codes[0]).shape[-2]
@@ -272,8 +276,8 @@ def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorO
 def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: TensorOrList,
                    w_scales_c: TensorOrList, offsets: torch.Tensor, status: torch.Tensor,
                    dx: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """dgrad on MXFP8 operands: dy rowwise codes [M,N] + k-group scales; W
-    columnwise codes [G,N,K] + columnwise scales."""
+    """dgrad on MXFP8 operands: dy rowwise codes [M,N] + scale atoms; W
+    columnwise codes [G,N,K] + columnwise scale atoms."""
     G = offsets.numel() - 1
     M, N = dy_codes.shape
     K = (w_codes_c if isinstance(w_codes_c, torch.Tensor) else w_codes_c[0]).shape[-1]
@@ -291,7 +295,7 @@ def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: T
 def gl_wgrad_mxfp8(x_codes_c: torch.Tensor, x_scales_c: torch.Tensor, dy_codes_c: torch.Tensor,
                    dy_scales_c: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
                    main_grad: TensorOrList, accumulate: bool = True) -> TensorOrList:
-    """wgrad on MXFP8 operands: x and dy columnwise codes + columnwise scales."""
+    """wgrad on MXFP8 operands: x and dy columnwise codes + columnwise scale atoms."""
     G = offsets.numel() - 1
     M, K = x_codes_c.shape
     N = dy_codes_c.shape[1]

@@ -83,11 +83,11 @@ const char* gl_status_string(gl_status s);
 
 /*
  * gl_set_cta_pair -- tile shape of the grouped GEMMs launched afterwards by
- * this process.  With GL_PAIRS_BF16 set (default) the bf16 GEMMs compute
- * 256 x 256 output tiles on pairs of CTAs (tcgen05 cta_group::2, one CTA per
- * SM), else 128 x 256 tiles on single CTAs.  With GL_PAIRS_MXFP8 set the
- * MXFP8 GEMMs compute 256 x 224 tiles on CTA pairs, else (default) 128 x 224
- * tiles on single CTAs.  Results agree within rounding.  Returns
+ * this process.  With GL_PAIRS_BF16 set the bf16 GEMMs compute 256 x 256
+ * output tiles on pairs of CTAs (tcgen05 cta_group::2, one CTA per SM), else
+ * 128 x 256 tiles on single CTAs.  With GL_PAIRS_MXFP8 set the MXFP8 GEMMs
+ * compute 256 x 192 tiles on CTA pairs, else 128 x 192 tiles on single CTAs.
+ * Both flags are set by default.  Results agree within rounding.  Returns
  * GL_ERR_INVALID for unknown flag bits.
  */
 #define GL_PAIRS_BF16 1
@@ -189,25 +189,47 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
  *   status      device int32 status word or NULL; non-zero -> nothing written
  *   codes_r     NULL or device u8 [rows, cols]: rowwise codes (blocks of 32
  *               along each row)
- *   scales_r    device u8 (required with codes_r): with scale_layout ==
- *               GL_SCALES_ROWMAJOR a [rows, cols/32] array; with
- *               GL_SCALES_KGROUP (cols % 128 == 0) a [cols/128][P][4] array,
- *               P = rows rounded up to a multiple of 4, whose element
- *               (j, r, b) is the scale of k-block 4j+b of row r -- the form
- *               the MXFP8 GEMMs read (one contiguous box per stage)
+ *   scales_r    device u8 (required with codes_r), in scale_layout:
+ *               GL_SCALES_ROWMAJOR: a [rows, cols/32] array;
+ *               GL_SCALES_MMA (cols % 128 == 0): 512-byte atoms, atom (q, b)
+ *               at byte (q * R + b) * 512 with R = ceil(rows/128), holding the
+ *               scales of k-blocks 4q..4q+3 of rows 128b..128b+127; the scale
+ *               of k-block 4q+j of row 128b+i sits at byte
+ *               (i % 32) * 16 + (i / 32) * 4 + j of its atom (the tcgen05
+ *               scale-factor layout, so the MXFP8 GEMMs copy atoms to tensor
+ *               memory as they are).  R * (cols/128) atoms.
  *   codes_c     NULL or device u8 [rows, cols]: columnwise codes (blocks of 32
  *               rows along each column, restarting at every group's first
  *               row; a group's last block may be partial)
- *   scales_c    device u8 [S, cols] (required with codes_c), where group i's
- *               block j is scale row sum_{l<i} ceil(m_l/32) + j;
- *               S <= ceil(rows/32) + G bounds the rows used.
+ *   scales_c    device u8 (required with codes_c), in scale_layout:
+ *               GL_SCALES_ROWMAJOR: [S, cols], group i's block j in scale
+ *               row sum_{l<i} ceil(m_l/32) + j, S <= ceil(rows/32) + G;
+ *               GL_SCALES_MMA (cols % 128 == 0): group i owns k-groups
+ *               T_i .. T_i + ceil(m_i/128) - 1, T_i = sum_{l<i} ceil(m_l/128);
+ *               atom (T_i + t, c) at byte ((T_i + t) * (cols/128) + c) * 512
+ *               holds blocks 4t..4t+3 of group i for columns 128c..128c+127,
+ *               the scale of block 4t+j of column 128c+n at byte
+ *               (n % 32) * 16 + (n / 32) * 4 + j.  At most
+ *               (ceil(rows/128) + G) * (cols/128) atoms.
+ *               In either MMA layout the bytes of rows (or blocks) that do not
+ *               exist are not written.
+ * gl_mxfp8_scale_bytes gives the bytes to allocate for a scale array.
  * Limits: cols % 32 == 0; rows/G integral when row_offsets is NULL.
  */
 #define GL_SCALES_ROWMAJOR 0
-#define GL_SCALES_KGROUP 1
+#define GL_SCALES_MMA 1
 gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                                int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                                uint8_t* codes_c, uint8_t* scales_c, int scale_layout, void* stream);
+
+/*
+ * gl_mxfp8_scale_bytes -- bytes of a scale array written by
+ * group_quantize_mxfp8 for a [rows, cols] source in G groups: rowwise
+ * (colwise == 0) or columnwise (colwise != 0) scales in scale_layout.  For
+ * columnwise scales with row offsets it is the bound that holds for any split
+ * sizes.  Host-only, no device access; returns 0 for invalid arguments.
+ */
+size_t gl_mxfp8_scale_bytes(int64_t rows, int cols, int G, int colwise, int scale_layout);
 
 /*
  * MXFP8 grouped GEMMs -- the three products of gl_fwd / gl_dgrad / gl_wgrad
@@ -220,16 +242,15 @@ gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const in
  * Outputs, offsets, status, caller buffers and main_grad behave exactly as in
  * the bf16 entry points.
  *
- * Operand forms (all device memory, produced by group_quantize_mxfp8):
+ * Operand forms (all device memory, produced by group_quantize_mxfp8; every
+ * scale array in the GL_SCALES_MMA layout):
  *   rowwise codes    u8 [rows, cols] (x, dy: [M, K] / [M, N]; W: [G, N, K])
- *   k-group scales   GL_SCALES_KGROUP rowwise scales, [cols/128][P][4] with
- *                    P = rows rounded up to 4 (x: cols K, rows M; dy: cols N,
- *                    rows M; stacked W: cols K, rows G*N; per-group W: rows N)
+ *   rowwise scales   x: rows M, cols K; dy: rows M, cols N; stacked W: rows
+ *                    G*N, cols K; per-group W: rows N, cols K
  *   columnwise codes u8 [rows, cols] (x_c [M, K], dy_c [M, N], W_c [G, N, K])
- *   columnwise scales u8 [S, cols] as group_quantize_mxfp8 writes them: for
- *                    x_c / dy_c quantized with the group offsets, S >=
- *                    ceil(M/32) + G rows allocated; for W_c (equal groups of
- *                    N rows) G * ceil(N/32) rows, or ceil(N/32) per group.
+ *   columnwise scales x_c / dy_c quantized with the group offsets; stacked
+ *                    W_c as G equal groups of N rows; per-group W_c as one
+ *                    group of N rows
  * Limits: N % 128 == 0, K % 128 == 0, G <= GL_MAX_GROUPS_MXFP8.
  */
 #define GL_MAX_GROUPS_MXFP8 2048

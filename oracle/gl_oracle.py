@@ -297,17 +297,53 @@ def quantize_rowwise(src: np.ndarray):
     return codes.reshape(rows, cols), (e + 127).astype(np.uint8)
 
 
-def rowwise_scales_kgroup(scales: np.ndarray) -> np.ndarray:
-    """Rowwise scales [rows, cols/32] rearranged k-group-major: element
-    (j, r, b) = scales[r, 4j + b], shape [cols/128, rows, 4] (the library pads
-    the row dimension to a multiple of 4; padding is not compared)."""
-    rows, nb = scales.shape
-    assert nb % 4 == 0
-    out = np.zeros((nb // 4, rows, 4), dtype=np.uint8)
-    for j in range(nb // 4):
-        for b in range(4):
-            out[j, :, b] = scales[:, 4 * j + b]
-    return out
+MMA_ATOM_BYTES = 512  # 128 operand rows x 4 blocks of 32 contraction elements
+
+
+def mma_atom_byte(i: int, j: int) -> int:
+    """Byte of operand row i (0..127) and block j (0..3) inside one 512-byte
+    scale atom of the tcgen05 block-scaled MMA: 32 lines of 16 bytes; line
+    i % 32 holds rows i, i+32, i+64, i+96 (4 bytes each, one per block)."""
+    return (i % 32) * 16 + (i // 32) * 4 + j
+
+
+def mma_offsets_rowwise(rows: int, cols: int) -> np.ndarray:
+    """Byte offset of every rowwise scale [rows, cols/32] in the MMA layout.
+
+    Atom (q, b) -- k-blocks 4q..4q+3 of rows 128b..128b+127 -- starts at
+    byte (q * R + b) * 512, R = ceil(rows / 128) (k-group-major, so one
+    k-group of consecutive row blocks is contiguous)."""
+    assert cols % 128 == 0
+    R = (rows + 127) // 128
+    off = np.empty((rows, cols // MX_BLOCK), dtype=np.int64)
+    for r in range(rows):
+        for k in range(cols // MX_BLOCK):
+            atom = (k // 4) * R + r // 128
+            off[r, k] = atom * MMA_ATOM_BYTES + mma_atom_byte(r % 128, k % 4)
+    return off
+
+
+def mma_offsets_colwise(m_splits, cols: int) -> np.ndarray:
+    """Byte offset of every columnwise scale [S, cols] (S = colwise_scale_rows
+    total; row base_i + j = block j of group i) in the MMA layout.
+
+    Group i owns k-groups T_i .. T_i + ceil(m_i/128) - 1 with
+    T_i = sum_{l<i} ceil(m_l / 128); k-group T_i + t holds the group's blocks
+    4t..4t+3; atom (T_i + t, c) -- columns 128c..128c+127 -- starts at byte
+    ((T_i + t) * cols/128 + c) * 512."""
+    assert cols % 128 == 0
+    C = cols // 128
+    base = colwise_scale_rows(m_splits)
+    off = np.empty((int(base[-1]), cols), dtype=np.int64)
+    T = 0
+    for i, m in enumerate(m_splits):
+        nblk = int(base[i + 1] - base[i])
+        for j in range(nblk):
+            kq = T + j // 4
+            for n in range(cols):
+                off[base[i] + j, n] = (kq * C + n // 128) * MMA_ATOM_BYTES + mma_atom_byte(n % 128, j % 4)
+        T += (int(m) + 127) // 128
+    return off
 
 
 def colwise_scale_rows(m_splits) -> np.ndarray:

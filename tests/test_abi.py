@@ -15,7 +15,7 @@ def _declared():
     with open(os.path.join(ROOT, "include", "gl.h")) as f:
         src = f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:gl_status|int|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:gl_status|int|size_t|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -61,6 +61,21 @@ def test_host_side_validation_without_gpu():
     # k-group-major scales need cols % 128 == 0; unknown layout codes are rejected
     assert lib.group_quantize_mxfp8(16, 8, 96, None, 1, None, 16, 16, None, None, 1, None) == gl.GL_ERR_UNSUPPORTED
     assert lib.group_quantize_mxfp8(16, 8, 128, None, 1, None, 16, 16, None, None, 7, None) == gl.GL_ERR_INVALID
+
+
+def test_scale_bytes_helper():
+    """Sizes of the scale arrays (host only): row-major [rows, cols/32] and
+    [ceil(rows/32) + G, cols]; MMA layout in 512-byte atoms of 128 rows x 4
+    blocks, columnwise bounded by ceil(rows/128) + G k-groups."""
+    lib = gl.load()
+    assert lib.gl_mxfp8_scale_bytes(100, 64, 3, 0, gl.GL_SCALES_ROWMAJOR) == 100 * 2
+    assert lib.gl_mxfp8_scale_bytes(100, 64, 3, 1, gl.GL_SCALES_ROWMAJOR) == (4 + 3) * 64
+    assert lib.gl_mxfp8_scale_bytes(300, 256, 3, 0, gl.GL_SCALES_MMA) == 3 * 2 * 512
+    assert lib.gl_mxfp8_scale_bytes(300, 256, 3, 1, gl.GL_SCALES_MMA) == (3 + 3) * 2 * 512
+    assert lib.gl_mxfp8_scale_bytes(300, 96, 3, 0, gl.GL_SCALES_MMA) == 0   # cols % 128 != 0
+    assert lib.gl_mxfp8_scale_bytes(300, 256, 0, 0, gl.GL_SCALES_MMA) == 0  # G <= 0
+    assert lib.gl_mxfp8_scale_bytes(300, 256, 1, 0, 5) == 0                 # unknown layout
+    assert lib.gl_mxfp8_scale_bytes(0, 128, 1, 1, gl.GL_SCALES_MMA) == 1 * 512
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

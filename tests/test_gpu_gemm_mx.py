@@ -32,9 +32,9 @@ TOL_MX = 1e-2
 def _quantize_all(d, m, G, N, K, off, st):
     """GPU MXFP8 copies of x, W and dy in the forms the GEMMs read."""
     q = {}
-    q["x"] = gl.group_quantize_mxfp8(d["x"], off, rowwise=True, colwise=True, status=st, kgroup_scales=True)
-    q["dy"] = gl.group_quantize_mxfp8(d["dy"], off, rowwise=True, colwise=True, status=st, kgroup_scales=True)
-    q["w"] = gl.group_quantize_mxfp8(d["w"], rowwise=True, colwise=True, kgroup_scales=True)  # G equal groups
+    q["x"] = gl.group_quantize_mxfp8(d["x"], off, rowwise=True, colwise=True, status=st, mma_scales=True)
+    q["dy"] = gl.group_quantize_mxfp8(d["dy"], off, rowwise=True, colwise=True, status=st, mma_scales=True)
+    q["w"] = gl.group_quantize_mxfp8(d["w"], rowwise=True, colwise=True, mma_scales=True)  # G equal groups
     return q
 
 
@@ -60,6 +60,7 @@ SMALL = [
     (1, 256, 256, [300]),
     (8, 128, 256, [1, 15, 17, 63, 64, 65, 0, 130]),
     (3, 512, 384, [257, 0, 511]),
+    (2, 896, 128, [200, 70]),  # five B tiles, starting 0 or 64 rows into a scale atom
 ]
 
 
@@ -71,13 +72,13 @@ def test_mxfp8_small(G, N, K, m, per_group, tile_mode):
     off, st = offsets_on_device(m, M, M + 32)
     q = _quantize_all(d, m, G, N, K, off, st)
     if per_group:
-        wc = [q["w"]["codes_r"][g * N:(g + 1) * N].contiguous() for g in range(G)]
-        # per-group k-group scales: [K/128, pitch(N), 4] for each group
-        ws_full = q["w"]["scales_r"]
-        ws = [ws_full[:, g * N:(g + 1) * N].contiguous() for g in range(G)]
-        wcc = [q["w"]["codes_c"][g * N:(g + 1) * N].contiguous() for g in range(G)]
-        n32 = (N + 31) // 32
-        wcs = [q["w"]["scales_c"][g * n32:(g + 1) * n32].contiguous() for g in range(G)]
+        # each weight quantized as its own [N, K] tensor: separate buffers per group
+        qg = [gl.group_quantize_mxfp8(d["w"][g].contiguous(), rowwise=True, colwise=True, mma_scales=True)
+              for g in range(G)]
+        wc = [t["codes_r"] for t in qg]
+        ws = [t["scales_r"] for t in qg]
+        wcc = [t["codes_c"] for t in qg]
+        wcs = [t["scales_c"] for t in qg]
         bias = [d["bias"][g].clone() for g in range(G)]
     else:
         wc = q["w"]["codes_r"].view(G, N, K)
@@ -113,6 +114,42 @@ def test_mxfp8_small(G, N, K, m, per_group, tile_mode):
         assert orc.rel_frobenius(got_w[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad", g)
         assert orc.rel_frobenius(got_a[g] - mg0[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad acc", g)
     assert untouched(y[M:]) and untouched(dx[M:])
+
+
+def test_mxfp8_many_groups_per_group(tile_mode):
+    """70 groups with per-group weights and main_grad: the launches cover 64
+    groups each, so the second one starts at a group whose scale k-groups
+    follow those of all earlier groups."""
+    G, N, K = 70, 128, 128
+    rng = np.random.default_rng(70)
+    m = [int(v) for v in rng.integers(0, 90, size=G)]
+    m[3] = m[64] = 0
+    M = sum(m)
+    d = {k: v.cuda() for k, v in synth.operands(G, M, N, K, seed=70, bias=True).items()}
+    off, st = offsets_on_device(m, M)
+    q = _quantize_all(d, m, G, N, K, off, st)
+    qg = [gl.group_quantize_mxfp8(d["w"][g].contiguous(), rowwise=True, colwise=True, mma_scales=True)
+          for g in range(G)]
+    y = gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], [t["codes_r"] for t in qg],
+                        [t["scales_r"] for t in qg], [d["bias"][g].clone() for g in range(G)], off, st)
+    dx = gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], [t["codes_c"] for t in qg],
+                           [t["scales_c"] for t in qg], off, st)
+    mg = torch.full((G, N, K), float("nan"), device="cuda")
+    gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
+                      [mg[g] for g in range(G)], accumulate=False)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = _oracle_all(d, m, G, N, K)
+    o = orc.offsets(m)
+    got_y, got_dx, got_w = f64(y), f64(dx), f64(mg)
+    for g in range(G):
+        a, b = int(o[g]), int(o[g + 1])
+        if a == b:
+            assert np.all(got_w[g] == 0.0)
+            continue
+        assert orc.rel_frobenius(got_y[a:b], ref["fwd"][a:b]) <= TOL_MX, ("fwd", g)
+        assert orc.rel_frobenius(got_dx[a:b], ref["dgrad"][a:b]) <= TOL_MX, ("dgrad", g)
+        assert orc.rel_frobenius(got_w[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad", g)
 
 
 def test_mxfp8_integer_mode_bit_exact(tile_mode):

@@ -41,18 +41,39 @@ def test_ragged_groups_bit_exact(m, cols):
     _check(src, m, got)
 
 
-@pytest.mark.parametrize("m,cols", [([0, 96, 160, 256], 128), ([5, 123, 0, 2], 384)])
-def test_kgroup_rowwise_scales(m, cols):
-    """The k-group-major rowwise scale layout holds the same bytes, permuted."""
+@pytest.mark.parametrize("m,cols", [([0, 96, 160, 256], 128), ([5, 123, 0, 2], 384), ([130, 1, 257], 256)])
+def test_mma_layout_scales(m, cols):
+    """Scales in the tcgen05 scale-factor layout: every byte the oracle places
+    (its own offset functions) equals the oracle's scale; codes unchanged."""
     rows = sum(m)
-    src = torch.randn(rows, cols, generator=torch.Generator().manual_seed(cols)).to(torch.bfloat16).cuda()
+    g = torch.Generator().manual_seed(cols + rows)
+    scale = torch.exp(torch.empty(rows, 1).uniform_(-6, 6, generator=g))
+    src = (torch.randn(rows, cols, generator=g) * scale).to(torch.bfloat16).cuda()
     off, st = gl.gl_offsets(torch.tensor(m, dtype=torch.int64, device="cuda"), rows)
-    got = gl.group_quantize_mxfp8(src, off, rowwise=True, colwise=False, status=st, kgroup_scales=True)
+    got = gl.group_quantize_mxfp8(src, off, rowwise=True, colwise=True, status=st, mma_scales=True)
     torch.cuda.synchronize()
+    assert got["scales_r"].numel() == ((rows + 127) // 128) * (cols // 128) * 512
+    assert got["scales_c"].numel() == ((rows + 127) // 128 + len(m)) * (cols // 128) * 512
     c, s = orc.quantize_rowwise(f64(src))
     assert np.array_equal(got["codes_r"].cpu().numpy(), c)
-    assert got["scales_r"].shape == (cols // 128, gl.kgroup_pitch(rows), 4)
-    assert np.array_equal(got["scales_r"][:, :rows].cpu().numpy(), orc.rowwise_scales_kgroup(s))
+    assert np.array_equal(got["scales_r"].cpu().numpy()[orc.mma_offsets_rowwise(rows, cols)], s)
+    cc, sc = orc.quantize_colwise(f64(src), m)
+    assert np.array_equal(got["codes_c"].cpu().numpy(), cc)
+    assert np.array_equal(got["scales_c"].cpu().numpy()[orc.mma_offsets_colwise(m, cols)], sc)
+
+
+def test_mma_layout_equal_groups():
+    """A stacked weight (equal groups, no offsets array) in the MMA layout:
+    member i owns k-groups i * ceil(rows_i / 128) onwards."""
+    G, R, C = 3, 256, 256
+    w = torch.randn(G, R, C, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16).cuda()
+    got = gl.group_quantize_mxfp8(w, rowwise=True, colwise=True, mma_scales=True)
+    torch.cuda.synchronize()
+    src = f64(w.reshape(G * R, C))
+    _, s = orc.quantize_rowwise(src)
+    assert np.array_equal(got["scales_r"].cpu().numpy()[orc.mma_offsets_rowwise(G * R, C)], s)
+    _, sc = orc.quantize_colwise(src, [R] * G)
+    assert np.array_equal(got["scales_c"].cpu().numpy()[orc.mma_offsets_colwise([R] * G, C)], sc)
 
 
 def test_every_bf16_value_bit_exact():

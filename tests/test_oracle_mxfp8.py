@@ -230,10 +230,51 @@ def test_planted_scale_mistake_is_caught():
     assert diffs > 0
 
 
-def test_kgroup_layout_is_a_permutation():
-    rng = np.random.default_rng(5)
-    sc = rng.integers(0, 256, (7, 12)).astype(np.uint8)
-    kg = orc.rowwise_scales_kgroup(sc)
-    assert kg.shape == (3, 7, 4)
-    assert sorted(kg.ravel().tolist()) == sorted(sc.ravel().tolist())
-    assert kg[2, 5, 1] == sc[5, 9] and kg[0, 0, 3] == sc[0, 3]
+def test_mma_rowwise_offsets_hand_worked():
+    """Positions worked by hand from the tcgen05 scale-factor layout (rows i,
+    i+32, i+64, i+96 of an atom share a 16-byte line, one byte per block;
+    atoms k-group-major): rows=300 (R = 3 row atoms), cols=256 (2 k-groups)."""
+    off = orc.mma_offsets_rowwise(300, 256)
+    assert off.shape == (300, 8)
+    assert off[0, 0] == 0
+    assert off[1, 0] == 16
+    assert off[32, 0] == 4
+    assert off[33, 2] == 16 + 4 + 2
+    assert off[127, 3] == 31 * 16 + 3 * 4 + 3
+    assert off[128, 0] == 512            # second row atom of k-group 0
+    assert off[0, 4] == 3 * 512          # k-group 1 starts after R = 3 atoms
+    assert off[299, 7] == 5 * 512 + 11 * 16 + 1 * 4 + 3   # row 299 = atom 2, i = 43
+
+
+def test_mma_colwise_offsets_hand_worked():
+    """Groups [100, 0, 300] x 128 columns: k-group bases T = [0, 1, 1]."""
+    off = orc.mma_offsets_colwise([100, 0, 300], 128)
+    base = orc.colwise_scale_rows([100, 0, 300])
+    assert off.shape == (int(base[-1]), 128)
+    assert off[base[0] + 3, 5] == 5 * 16 + 0 * 4 + 3          # group 0, block 3 (rows 96..99)
+    assert off[base[2] + 0, 0] == 512                          # group 2 starts k-group 1
+    assert off[base[2] + 9, 127] == 3 * 512 + 31 * 16 + 3 * 4 + 1  # block 9 -> k-group 1 + 2, j = 1
+    assert off[base[2] + 4, 64] == 2 * 512 + 0 * 16 + 2 * 4 + 0
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (130, 256), (300, 384)])
+def test_mma_rowwise_offsets_injective_in_bounds(rows, cols):
+    off = orc.mma_offsets_rowwise(rows, cols)
+    bound = ((rows + 127) // 128) * (cols // 128) * 512
+    assert len(np.unique(off)) == off.size
+    assert off.min() >= 0 and off.max() < bound
+
+
+@pytest.mark.parametrize("m", [[1], [100, 0, 300], [128, 129, 127, 33], [0, 0, 5]])
+def test_mma_colwise_offsets_injective_in_bounds(m):
+    cols = 256
+    off = orc.mma_offsets_colwise(m, cols)
+    rows, G = sum(m), len(m)
+    bound = ((rows + 127) // 128 + G) * (cols // 128) * 512
+    assert len(np.unique(off)) == off.size
+    assert off.min() >= 0 and off.max() < bound
+    # one group alone lands in the rowwise layout of its transpose
+    if len(m) == 1:
+        t = orc.mma_offsets_rowwise(cols, ((m[0] + 127) // 128) * 128)
+        nblk = (m[0] + 31) // 32
+        assert np.array_equal(off, t[:, :nblk].T)
