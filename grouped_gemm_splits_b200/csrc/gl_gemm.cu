@@ -477,6 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t r[32];
           tmem_ld_32x32b_x32(tacc + c * 32, r);
           tmem_ld_wait();
+          tmem_reg_fence(r);
           if (c == nchunks - 1) release_acc();  // accumulator fully read
           float v[32];
 #pragma unroll
@@ -524,6 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (have_acc) {
             tmem_ld_32x32b_x32(tacc + c * 32, r);
             tmem_ld_wait();
+            tmem_reg_fence(r);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) r[j] = 0u;

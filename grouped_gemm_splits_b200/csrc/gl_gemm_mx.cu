@@ -7,11 +7,14 @@
 // columnwise for wgrad), computed as sum_k (q_a 2^sa)(q_b 2^sb) by
 // tcgen05.mma kind::mxf8f6f4.block_scale with fp32 accumulation in TMEM.
 //
-// Output tile 128*CG x 192.  With CG = 2 a cluster pair shares the tile
-// (tcgen05 cta_group::2): each CTA loads its own 128 rows of A and 96 rows
+// Output tile 128*CG x TN.  With CG = 2 a cluster pair shares the tile
+// (tcgen05 cta_group::2): each CTA loads its own 128 rows of A and TN/2 rows
 // of B; the peer relays "stage landed" to the leader, which issues the MMAs.
-// Two 192-column fp32 accumulators (384 TMEM columns) leave 128 columns for
-// the scale-factor slots.
+// fprop / dgrad: TN = 256 and one fp32 accumulator (256 TMEM columns); eight
+// epilogue warps copy it to registers and free it at once, so the next tile's
+// MMAs overlap the stores.  wgrad: TN = 192 and two accumulators (384
+// columns); four epilogue warps stage fp32 boxes for TMA reduce-adds.  The
+// remaining TMEM columns hold the scale-factor slots.
 //
 // Per stage (128 contraction elements = four MMAs of K=32) the producer
 // TMA-loads the codes (128-byte swizzle) and the scales.  The scales arrive
@@ -19,12 +22,12 @@
 // scale-factor layout (128 operand rows x 4 blocks; row i at byte
 // (i%32)*16 + ((i/32)%4)*4 + block), so a stage's scales are two plain boxes:
 // one atom for the CTA's 128 A rows and two consecutive atoms (256 rows)
-// covering the tile's 192 B rows.  The MMA thread copies them to TMEM with
+// covering the tile's B rows.  The MMA thread copies them to TMEM with
 // tcgen05.cp.32x128b.warpx4 and selects scale byte kb of each MMA through the
 // instruction descriptor.  B row i of a tile that starts at operand row
 // 128c + 32s reads TMEM column (slot + s) + i/32, so the MMA's scale address is
-// offset by s columns; with 192-row tiles s is 0 or 2 (tiles start on
-// multiples of 64 rows).  A tiles (fprop / dgrad) start on 128-row boundaries of
+// offset by s columns: 0 for 256-row tiles, 0 or 2 for 192-row tiles (their
+// starts are multiples of 64 rows).  A tiles (fprop / dgrad) start on 128-row boundaries of
 // the packed activations: a group's first tile may begin inside the previous
 // group, and only the group's own rows are stored.
 //
@@ -45,29 +48,32 @@ namespace gl {
 namespace {
 
 constexpr int BK = 128;  // fp8 contraction elements per stage (128 bytes)
-constexpr int TN = 192;  // accumulator columns (tile starts on multiples of 64 B rows)
-constexpr int kThreads = 192;  // warp 0 TMA, 1 MMA (leader) / relay (peer), 2-5 epilogue
 constexpr int kPG = 64;
 constexpr int kBand = 8;
-constexpr int kSfCol0 = 2 * TN;  // first TMEM column of the scale-factor slots
 constexpr int kSfSlots = 4;      // slot j: A at +0 (4 columns), B at +4 (8 columns)
 constexpr int kSfSlotCols = 16;
 constexpr int kSfABytes = 512;   // one atom
-constexpr int kAtomsB = 2;       // 256 B rows cover a 192-row tile starting 0 or 64 rows into an atom
+constexpr int kAtomsB = 2;       // 256 B rows: a whole 256-row tile, or a 192-row tile 0 or 64 rows in
 constexpr int kSfBytes = 2048;   // A atom + B atoms, padded to keep stages 1 KB aligned
 static_assert(kSfABytes + kAtomsB * 512 <= kSfBytes, "scale staging");
-static_assert((TN % 64) == 0 && 64 + TN <= 128 * kAtomsB, "B tile must stay inside the loaded atoms");
 
 template <int MODE, int CG>
 struct CfgMX {
+  static constexpr int kTN = (MODE == kWgrad) ? 192 : 256;  // accumulator columns
+  static constexpr int kAccBufs = (MODE == kWgrad) ? 2 : 1;
+  static constexpr int kEpiWarps = (MODE == kWgrad) ? 4 : 8;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, 1 MMA / relay, then epilogue
+  static constexpr int kSfCol0 = kAccBufs * kTN;        // first TMEM column of the scale-factor slots
   static constexpr int kTileM = 128 * CG;
-  static constexpr int kBRows = TN / CG;  // B rows held per CTA (192 or 96)
+  static constexpr int kBRows = kTN / CG;  // B rows held per CTA
   static constexpr int kABytes = 128 * BK;  // 16 KB
   // B codes per CTA: K-major kBRows x 128 B, MN-major 128-column chunks
-  static constexpr int kBChunks = (CG == 1 ? 2 : 1);
-  static constexpr int kBAlloc = kBChunks * 128 * BK;
-  static constexpr int kBLoad = (MODE == kFwd) ? kBRows * BK : kBAlloc;
-  static constexpr int kStageBytes = kABytes + kBAlloc + kSfBytes;  // 50 KB / 34 KB
+  static constexpr int kBChunks = (kBRows + 127) / 128;
+  static constexpr int kBAlloc = (MODE == kFwd) ? kBRows * BK : kBChunks * 128 * BK;
+  static constexpr int kBLoad = kBAlloc;
+  static_assert((kTN % 128 == 0 ? 0 : 64) + kTN <= 128 * kAtomsB && kTN % 64 == 0,
+                "B tile must stay inside the loaded scale atoms");
+  static constexpr int kStageBytes = kABytes + kBAlloc + kSfBytes;  // 50 KB (CG 1) / 34 KB (CG 2)
   static constexpr int kStagingBytes = (MODE == kWgrad) ? 4 * 2 * 32 * 32 * 4 : 0;
   static constexpr int kStages = CG == 2 ? ((MODE == kWgrad) ? 5 : 6) : ((MODE == kWgrad) ? 3 : 4);
   static constexpr int kTx = kABytes + kBLoad + kSfABytes + kAtomsB * 512;
@@ -133,7 +139,7 @@ __device__ __forceinline__ int64_t atom_floor(int64_t r) { return r & ~int64_t(1
 
 template <int MODE, int CG>
 __device__ __forceinline__ int tiles_of_group(int64_t o0, int64_t o1, const MxParams& p) {
-  constexpr int TMt = CfgMX<MODE, CG>::kTileM;
+  constexpr int TMt = CfgMX<MODE, CG>::kTileM, TN = CfgMX<MODE, CG>::kTN;
   const int64_t m = o1 > o0 ? o1 - o0 : 0;
   if (MODE == kWgrad) return (m > 0 || !p.accumulate) ? cdiv(p.N, TMt) * cdiv(p.K, TN) : 0;
   if (m == 0) return 0;
@@ -142,7 +148,7 @@ __device__ __forceinline__ int tiles_of_group(int64_t o0, int64_t o1, const MxPa
 
 template <int MODE, int CG>
 __device__ __forceinline__ Tile decode(int t, const int* prefix, const MxParams& p) {
-  constexpr int TMt = CfgMX<MODE, CG>::kTileM;
+  constexpr int TMt = CfgMX<MODE, CG>::kTileM, TN = CfgMX<MODE, CG>::kTN;
   int lo = 0, hi = p.G;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -206,10 +212,10 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* sa, uint8_t* sb, int val
 }
 
 template <int MODE, int CG, bool PG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
     grouped_gemm_mx_kernel(const __grid_constant__ MxParams p, const __grid_constant__ MxPG<PG> pg) {
   using C = CfgMX<MODE, CG>;
-  constexpr int TMt = C::kTileM;
+  constexpr int TMt = C::kTileM, TN = C::kTN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4 * CG);
+      mbar_init(&tempty[b], C::kEpiWarps * CG);
     }
     mbar_init(mma_done, 1);
     fence_barrier_init();
@@ -383,8 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kiter = 0;
       for (int t = pair; t < total; t += npairs, ++it) {
         const Tile tl = decode<MODE, CG>(t, prefix, p);
-        const int buf = it & 1;
-        const uint32_t tph = (it >> 1) & 1;
+        const int buf = it % C::kAccBufs;
+        const uint32_t tph = (it / C::kAccBufs) & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], tph ^ 1u, abort_flag))) {
           report_abort(abort_flag, p.status);
           break;
@@ -418,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (MODE == kWgrad && valid < BK) zero_tail_rows<MODE, CG>(sa, sb, valid, ksteps * 32, lane);
           __syncwarp();
           if (lane == 0) {
-            const uint32_t sfa = tmem_base + kSfCol0 + (kiter & (kSfSlots - 1)) * kSfSlotCols;
+            const uint32_t sfa = tmem_base + C::kSfCol0 + (kiter & (kSfSlots - 1)) * kSfSlotCols;
             const uint32_t sfb0 = sfa + 4;
             const uint32_t pa = smem_u32(sf), pb = smem_u32(sf + kSfABytes);
             if (CG == 2) {
@@ -500,16 +506,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ===================== epilogue (warps 2..5, both CTAs) =====================
-    const int q = warp & 3;
+    // ===================== epilogue (warps 2.., both CTAs) =====================
+    const int q = warp & 3;                // TMEM lane quarter this warp may access
+    const int h = (warp - 2) >> 2;         // FWD/DGRAD: 128-column half of the tile
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_leader = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : 0u;
     int it = 0;
     int chunk_ctr = 0;
     for (int t = pair; t < total; t += npairs, ++it) {
       const Tile tl = decode<MODE, CG>(t, prefix, p);
-      const int buf = it & 1;
-      const uint32_t tph = (it >> 1) & 1;
+      const int buf = it % C::kAccBufs;
+      const uint32_t tph = (it / C::kAccBufs) & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
       if (!ok) report_abort(abort_flag, p.status);
       if (!ok) break;
@@ -524,45 +531,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       if (MODE != kWgrad) {
+        // this warp: rows q*32.. of the CTA's 128, columns h*128 .. h*128+127;
+        // copy them to registers, free the accumulator, then round and store
         const int Nout = (MODE == kFwd) ? p.N : p.K;
         const int64_t row = tl.r0 + hr + row_in_tile;
         const bool row_ok = row >= tl.rlo && row < tl.r1 && row < p.out_rows;
+        const int ncol0 = tl.nt * TN + h * 128;
+        const int nvalid = Nout - ncol0;  // columns of this warp inside the output (may be <= 0)
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c * 32 < nvalid) tmem_ld_32x32b_x32(tacc + h * 128 + c * 32, r[c]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_reg_fence(r[c]);
+        release_acc();
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
         const __nv_bfloat16* bias = nullptr;
         if (MODE == kFwd && p.has_bias) bias = PG ? pg.b(tl.g) : (p.bias + static_cast<int64_t>(tl.g) * p.N);
-        const int nchunks = min(TN / 32, cdiv(Nout - tl.nt * TN, 32));
-        for (int c = 0; c < nchunks; ++c) {
-          const int n = tl.nt * TN + c * 32;
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tacc + c * 32, r);
-          tmem_ld_wait();
-          if (c == nchunks - 1) release_acc();
-          float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if (bias != nullptr) {
+        for (int c = 0; c < 4; ++c) {
+          if (c * 32 >= nvalid) break;
 #pragma unroll
-            for (int j8 = 0; j8 < 4; ++j8) {
-              if (n + j8 * 8 < Nout) {
-                const uint4 bv = __ldg(reinterpret_cast<const uint4*>(bias + n + j8 * 8));
-                const __nv_bfloat16* bb = reinterpret_cast<const __nv_bfloat16*>(&bv);
+          for (int j8 = 0; j8 < 4; ++j8) {
+            const int n = ncol0 + c * 32 + j8 * 8;  // 8 output columns (16 bytes)
+            if (n >= Nout) break;
+            float f[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j8 * 8 + j] += __bfloat162float(bb[j]);
-              }
+            for (int j = 0; j < 8; ++j) f[j] = __uint_as_float(r[c][j8 * 8 + j]);
+            if (bias != nullptr) {
+              const uint4 bv = __ldg(reinterpret_cast<const uint4*>(bias + n));
+              const __nv_bfloat16* bb = reinterpret_cast<const __nv_bfloat16*>(&bv);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) f[j] += __bfloat162float(bb[j]);
             }
-          }
-          if (row_ok) {
-            __nv_bfloat16* dst = out + row * static_cast<int64_t>(Nout) + n;
-#pragma unroll
-            for (int j8 = 0; j8 < 4; ++j8) {
-              if (n + j8 * 8 < Nout) {
-                uint4 w;
-                w.x = pack_bf16x2(v[j8 * 8 + 0], v[j8 * 8 + 1]);
-                w.y = pack_bf16x2(v[j8 * 8 + 2], v[j8 * 8 + 3]);
-                w.z = pack_bf16x2(v[j8 * 8 + 4], v[j8 * 8 + 5]);
-                w.w = pack_bf16x2(v[j8 * 8 + 6], v[j8 * 8 + 7]);
-                *reinterpret_cast<uint4*>(dst + j8 * 8) = w;
-              }
+            if (row_ok) {
+              uint4 w;
+              w.x = pack_bf16x2(f[0], f[1]);
+              w.y = pack_bf16x2(f[2], f[3]);
+              w.z = pack_bf16x2(f[4], f[5]);
+              w.w = pack_bf16x2(f[6], f[7]);
+              *reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(Nout) + n) = w;
             }
           }
         }
@@ -583,6 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (have_acc) {
             tmem_ld_32x32b_x32(tacc + c * 32, r);
             tmem_ld_wait();
+            tmem_reg_fence(r);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) r[j] = 0u;
@@ -654,10 +664,10 @@ constexpr int mx_smem_bytes(int G) {
   return CfgMX<MODE, CG>::kPrefixOffset + 2 * (G + 1) * 4 + 1024;
 }
 
-cudaLaunchConfig_t pair_cfg(int grid, int smem, cudaStream_t stream, cudaLaunchAttribute* attr) {
+cudaLaunchConfig_t pair_cfg(int grid, int threads, int smem, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -670,7 +680,7 @@ cudaLaunchConfig_t pair_cfg(int grid, int smem, cudaStream_t stream, cudaLaunchA
 }
 
 template <typename Kern>
-int pair_grid(Kern kern, int smem) {
+int pair_grid(Kern kern, int threads, int smem) {
   static std::mutex mu;
   static std::unordered_map<const void*, int> cache;
   int dev = 0;
@@ -682,7 +692,7 @@ int pair_grid(Kern kern, int smem) {
     if (it != cache.end()) return it->second;
   }
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_cfg(2 * (num_sms() / 2), smem, nullptr, attr);
+  cudaLaunchConfig_t cfg = pair_cfg(2 * (num_sms() / 2), threads, smem, nullptr, attr);
   int nclusters = 0;
   if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters <= 0)
     nclusters = num_sms() / 2;
@@ -697,11 +707,12 @@ gl_status mx_launch(const MxParams& prm, const MxPG<PG>& pga, int G, cudaStream_
   const int smem = mx_smem_bytes<MODE, CG>(G);
   auto kern = grouped_gemm_mx_kernel<MODE, CG, PG>;
   if (set_max_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return GL_ERR_CUDA;
+  constexpr int threads = CfgMX<MODE, CG>::kThreads;
   if (CG == 1) {
-    kern<<<num_sms(), kThreads, smem, stream>>>(prm, pga);
+    kern<<<num_sms(), threads, smem, stream>>>(prm, pga);
   } else {
     cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = pair_cfg(pair_grid(kern, smem), smem, stream, attr);
+    cudaLaunchConfig_t cfg = pair_cfg(pair_grid(kern, threads, smem), threads, smem, stream, attr);
     if (cudaLaunchKernelEx(&cfg, kern, prm, pga) != cudaSuccess) return GL_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
