@@ -284,7 +284,7 @@ gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, co
 }
 
 gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
-                               int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                               int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                                uint8_t* codes_c, uint8_t* scales_c, int scale_layout, void* stream) {
   if (src == nullptr || rows < 0 || cols <= 0 || G <= 0 || G > GL_MAX_GROUPS) return GL_ERR_INVALID;
   if (codes_r == nullptr && codes_c == nullptr) return GL_ERR_INVALID;

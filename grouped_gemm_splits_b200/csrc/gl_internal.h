@@ -74,7 +74,7 @@ gl_status launch_offsets(const int64_t* m, int G, int64_t expect_rows, int64_t o
                          int64_t* offsets, int32_t* status, cudaStream_t stream);
 
 gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
-                          int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                          int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                           uint8_t* codes_c, uint8_t* scales_c, int scale_layout, cudaStream_t stream);
 
 }  // namespace gl

@@ -9,16 +9,19 @@
 // PR #3224).
 //
 // Work unit: a 32-row block of one group (the columnwise block) x 256
-// columns.  Every element is read once (16-byte loads, a warp covers 512
-// contiguous bytes of a row); rowwise amax is a 4-lane shuffle reduction,
-// columnwise amax a shared-memory reduction over the block's 32 rows.  The
-// kernel is persistent; each CTA first builds the per-group block prefix in
-// shared memory.  Memory-bound: 2 bytes read and up to 2 bytes (+1/16 for
-// scales) written per element.
+// columns (16 KB of bf16).  The kernel is persistent; one thread of each CTA
+// keeps a ring of kQStages tiles loaded ahead by TMA (mbarrier completion),
+// and the CTA's 256 threads read each element once from shared memory (a
+// thread: 4 rows x 8 columns).  Rowwise amax is a 4-lane shuffle reduction,
+// columnwise amax a shared-memory reduction over the block's 32 rows.  Each
+// CTA first builds the per-group block prefixes in shared memory.
+// Memory-bound: 2 bytes read and up to 2 bytes (+1/16 for scales) written per
+// element.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
 #include "gl_internal.h"
+#include "gl_ptx.cuh"
 
 namespace gl {
 namespace {
@@ -26,176 +29,249 @@ namespace {
 constexpr int kQThreads = 256;
 constexpr int kQCols = 256;
 constexpr int kQRows = 32;
+constexpr int kQTileBytes = kQRows * kQCols * 2;  // one work unit of bf16
+static_assert(kQThreads == 256 && kQCols == 256, "one column per thread; 8 warps x 4 rows = 32 rows");
+constexpr int kQStages = 4;     // tiles staged in shared memory by TMA
+constexpr int kQCtasPerSm = 2;  // 2 x 4 x 16 KB of loads in flight per SM
 
-// Scale exponent: smallest e with amax <= 448 * 2^e, clamped to [-127, 127];
-// 448 = 1.75 * 2^8, so for amax = 1.f * 2^E the answer is E - 8, plus one when
-// 1.f > 1.75.  amax = 0 gives 0.
+// Scale exponent: the smallest e with amax <= 448 * 2^e, clamped to
+// [-127, 127].  448 = 1.75 * 2^8, so for amax = 1.m * 2^(E-127) the answer is
+// E - 135, plus one when 1.m > 1.75; a subnormal amax (E = 0) is below
+// 448 * 2^-127; amax = 0 gives 0.  Branch-free (selects only).
 __device__ __forceinline__ int mx_scale_exp(float amax) {
   const uint32_t b = __float_as_uint(amax);
-  const int E = static_cast<int>((b >> 23) & 0xFFu);
-  const uint32_t mant = b & 0x7FFFFFu;
-  int e;
-  if (amax == 0.0f) e = 0;
-  else if (E == 0) e = -127;  // subnormal amax: below 448 * 2^-127
-  else e = (E - 127) - 8 + (mant > 0x600000u ? 1 : 0);
-  return e < -127 ? -127 : (e > 127 ? 127 : e);
+  const int E = static_cast<int>(b >> 23);
+  const int e = max(E - 135 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0), -127);
+  return b == 0 ? 0 : e;
 }
 
-// 2^-e as a float (e in [-127, 126] gives a normal number).
+// 2^-e as a float; e in [-127, 120] (the range finite bf16 amax values give)
+// is a normal number.
 __device__ __forceinline__ float pow2_neg(int e) {
-  const int bexp = 127 - e;
-  return bexp >= 1 && bexp <= 254 ? __uint_as_float(static_cast<uint32_t>(bexp) << 23) : 0.0f;
+  return __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
 }
 
-__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
-  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
-  return lo | (hi << 16);
+// (a, b) * (sa, sb) with one packed fp32 multiply (exact here: the scales
+// are powers of two and the products stay in the normal range or round to
+// zero in E4M3 anyway), rounded to two E4M3 codes (satfinite), a in the low
+// byte.
+__device__ __forceinline__ uint32_t e4m3x2_scaled(float a, float b, float sa, float sb) {
+  uint16_t q;
+  asm("{\n\t.reg .b64 v, s, p;\n\t.reg .f32 x, y;\n\t"
+      "mov.b64 v, {%1, %2};\n\t"
+      "mov.b64 s, {%3, %4};\n\t"
+      "mul.rn.f32x2 p, v, s;\n\t"
+      "mov.b64 {x, y}, p;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 %0, y, x;\n\t}"
+      : "=h"(q)
+      : "f"(a), "f"(b), "f"(sa), "f"(sb));
+  return q;
 }
 
-__global__ void __launch_bounds__(kQThreads, 4)
-    quantize_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int cols,
-                    const int64_t* __restrict__ row_offsets, int G, const int32_t* __restrict__ status,
+// Eight values times their scales -> eight E4M3 codes (first value lowest).
+__device__ __forceinline__ uint2 e4m3x8(const float (&v)[8], const float (&sc)[8]) {
+  uint2 q;
+  q.x = e4m3x2_scaled(v[0], v[1], sc[0], sc[1]) | (e4m3x2_scaled(v[2], v[3], sc[2], sc[3]) << 16);
+  q.y = e4m3x2_scaled(v[4], v[5], sc[4], sc[5]) | (e4m3x2_scaled(v[6], v[7], sc[6], sc[7]) << 16);
+  return q;
+}
+
+// max |v| over eight values, as a balanced tree (short dependency chains).
+__device__ __forceinline__ float amax8(const float (&v)[8]) {
+  const float a = fmaxf(fabsf(v[0]), fabsf(v[1])), b = fmaxf(fabsf(v[2]), fabsf(v[3]));
+  const float c = fmaxf(fabsf(v[4]), fabsf(v[5])), d = fmaxf(fabsf(v[6]), fabsf(v[7]));
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
+    quantize_kernel(const __grid_constant__ CUtensorMap tm_src, int64_t rows, int cols, int box_rows,
+                    int tile_bytes, const int64_t* __restrict__ row_offsets, int G, int32_t* status,
                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r,
                     uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, int64_t scales_c_bytes,
                     int mma_layout) {
-  extern __shared__ int64_t qsmem[];
-  int64_t* bprefix = qsmem;        // G+1: first 32-row block of each group (ragged mode)
-  int64_t* qprefix = qsmem + G + 1;  // G+1: first 128-row k-group of each group (ragged mode)
-  __shared__ float cmax[kQThreads / 32][kQCols];
-  __shared__ float csf[kQCols];
-  if (status != nullptr && *status != 0) return;
+  extern __shared__ uint8_t qsmem_raw[];
+  uint8_t* qsmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_buf = qsmem;                                                  // kQStages x 16 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsmem + kQStages * kQTileBytes);  // one barrier per stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kQStages);
+  int64_t* bprefix = reinterpret_cast<int64_t*>(qsmem + kQStages * kQTileBytes + 64);  // G+1 (ragged)
+  int64_t* qprefix = bprefix + G + 1;                                                  // G+1 (ragged)
+  __shared__ __align__(16) float cmax[kQThreads / 32][kQCols];  // per-warp column maxima
+  __shared__ __align__(16) float csf[kQCols];                     // 2^-e of each column
+  if (status != nullptr && *reinterpret_cast<volatile int32_t*>(status) != 0) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
 
   const int64_t per = (row_offsets == nullptr) ? rows / G : 0;
   const int64_t bpg = (per + kQRows - 1) / kQRows;  // blocks per group (uniform mode)
   const int64_t qpg = (per + 127) / 128;            // k-groups per group (uniform mode)
   const int64_t mma_rb = (rows + 127) / 128;        // 128-row blocks (rowwise MMA layout)
   const int mma_cb = cols / 128;                    // 128-column blocks (columnwise MMA layout)
-  int64_t nblocks;
-  if (row_offsets != nullptr) {
-    if (warp == 0) {
-      int64_t carry = 0, qcarry = 0;
-      for (int base = 0; base < G; base += 32) {
-        const int i = base + lane;
-        int64_t cnt = 0, qc = 0;
-        if (i < G) {
-          const int64_t m = row_offsets[i + 1] - row_offsets[i];
-          cnt = m > 0 ? (m + kQRows - 1) / kQRows : 0;
-          qc = m > 0 ? (m + 127) / 128 : 0;
-        }
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int64_t u = __shfl_up_sync(0xffffffffu, cnt, off);
-          const int64_t w = __shfl_up_sync(0xffffffffu, qc, off);
-          if (lane >= off) { cnt += u; qc += w; }
-        }
-        if (i < G) { bprefix[i + 1] = carry + cnt; qprefix[i + 1] = qcarry + qc; }
-        carry += __shfl_sync(0xffffffffu, cnt, 31);
-        qcarry += __shfl_sync(0xffffffffu, qc, 31);
+  if (row_offsets != nullptr && warp == 0) {
+    int64_t carry = 0, qcarry = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int i = base + lane;
+      int64_t cnt = 0, qc = 0;
+      if (i < G) {
+        const int64_t m = row_offsets[i + 1] - row_offsets[i];
+        cnt = m > 0 ? (m + kQRows - 1) / kQRows : 0;
+        qc = m > 0 ? (m + 127) / 128 : 0;
       }
-      if (lane == 0) { bprefix[0] = 0; qprefix[0] = 0; }
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int64_t u = __shfl_up_sync(0xffffffffu, cnt, off);
+        const int64_t w = __shfl_up_sync(0xffffffffu, qc, off);
+        if (lane >= off) { cnt += u; qc += w; }
+      }
+      if (i < G) { bprefix[i + 1] = carry + cnt; qprefix[i + 1] = qcarry + qc; }
+      carry += __shfl_sync(0xffffffffu, cnt, 31);
+      qcarry += __shfl_sync(0xffffffffu, qc, 31);
     }
-    __syncthreads();
-    nblocks = bprefix[G];
-  } else {
-    nblocks = bpg * G;
+    if (lane == 0) { bprefix[0] = 0; qprefix[0] = 0; }
   }
+  __syncthreads();
+  const int64_t nblocks = (row_offsets != nullptr) ? bprefix[G] : bpg * G;
   const int ncc = (cols + kQCols - 1) / kQCols;
   const int64_t ntiles = nblocks * ncc;
   const int c8 = lane;         // 8-column chunk within the 256-column tile
   const int rbase = warp * 4;  // this thread's 4 rows within the 32-row block
+  const int pitch = tile_bytes / box_rows;  // bytes per staged row (2 * min(cols, 256))
 
-  // Where tile t lives: group g, block j, first row r0 and valid row count.
-  auto locate = [&](int64_t t, int& g, int64_t& j, int64_t& r0, int& vrows, int& cc) {
-    const int64_t rb = t / ncc;
-    cc = static_cast<int>(t - rb * ncc);
-    int64_t gstart, gend;
-    if (row_offsets != nullptr) {
-      int lo = 0, hi = G;
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (bprefix[mid] <= rb) lo = mid; else hi = mid;
-      }
-      g = lo;
-      j = rb - bprefix[g];
-      gstart = min(max(row_offsets[g], int64_t(0)), rows);  // clamp: never leave [0, rows)
-      gend = min(max(row_offsets[g + 1], gstart), rows);
+  // Tile t = rb * ncc + cc (rb: 32-row block, counted over all groups; cc:
+  // 256-column chunk).  A CTA visits t = blockIdx.x + k * gridDim.x; the
+  // position advances by (gridDim.x / ncc, gridDim.x % ncc) with a carry and
+  // the group index moves forward with it, so the loop does no 64-bit
+  // division.
+  const bool ragged = row_offsets != nullptr;
+  const int step_rb = static_cast<int>(gridDim.x) / ncc, step_cc = static_cast<int>(gridDim.x) % ncc;
+  struct Pos {
+    int64_t rb;
+    int cc, g;
+  };
+  auto advance_group = [&](Pos& q) {
+    if (ragged) {
+      while (q.g + 1 < G && bprefix[q.g + 1] <= q.rb) ++q.g;
     } else {
-      g = static_cast<int>(rb / bpg);
-      j = rb - static_cast<int64_t>(g) * bpg;
-      gstart = static_cast<int64_t>(g) * per;
+      while (q.g + 1 < G && static_cast<int64_t>(q.g + 1) * bpg <= q.rb) ++q.g;
+    }
+  };
+  auto step = [&](Pos& q) {
+    q.cc += step_cc;
+    q.rb += step_rb;
+    if (q.cc >= ncc) { q.cc -= ncc; ++q.rb; }
+    advance_group(q);
+  };
+  // Block j of group g, its first row r0 and valid row count.
+  auto resolve = [&](const Pos& q, int64_t& j, int64_t& r0, int& vrows) {
+    int64_t gstart, gend;
+    if (ragged) {
+      j = q.rb - bprefix[q.g];
+      gstart = min(max(row_offsets[q.g], int64_t(0)), rows);  // clamp: never leave [0, rows)
+      gend = min(max(row_offsets[q.g + 1], gstart), rows);
+    } else {
+      j = q.rb - static_cast<int64_t>(q.g) * bpg;
+      gstart = static_cast<int64_t>(q.g) * per;
       gend = gstart + per;
     }
     r0 = gstart + j * kQRows;
     vrows = static_cast<int>(max(int64_t(0), min(static_cast<int64_t>(kQRows), gend - r0)));
   };
-  // 16-byte loads of this thread's 4 rows x 8 columns of tile t (zeros outside)
-  auto fetch = [&](int64_t r0, int vrows, int cc, uint4 (&raw)[4]) {
-    const int col = cc * kQCols + c8 * 8;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = rbase + i;
-      if (col < cols && r < vrows)
-        raw[i] = __ldg(reinterpret_cast<const uint4*>(src + (r0 + r) * cols + col));
-      else
-        raw[i] = make_uint4(0, 0, 0, 0);
-    }
+  // Stage s <- the tile at q (rows of other groups and past the tensor are
+  // masked or zero-filled; the consumers use only the block's valid rows).
+  auto issue = [&](const Pos& q, int s) {
+    int64_t jq, rq;
+    int vq;
+    resolve(q, jq, rq, vq);
+    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(tile_bytes));
+    tma_load_2d(stage_buf + s * kQTileBytes, &tm_src, &full[s], q.cc * kQCols, static_cast<int32_t>(rq));
   };
 
   int64_t t = blockIdx.x;
-  int g = 0, vrows = 0, cc = 0;
-  int64_t j = 0, r0 = 0;
-  uint4 raw[4];
-  if (t < ntiles) {
-    locate(t, g, j, r0, vrows, cc);
-    fetch(r0, vrows, cc, raw);
+  Pos pos;
+  pos.rb = static_cast<int>(blockIdx.x) / ncc;
+  pos.cc = static_cast<int>(blockIdx.x) % ncc;
+  pos.g = 0;
+  if (ragged) {
+    int lo = 0, hi = G;  // last group whose first block is <= rb
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (bprefix[mid] <= pos.rb) lo = mid; else hi = mid;
+    }
+    pos.g = lo;
   }
-  for (; t < ntiles; t += gridDim.x) {
-    // issue the next tile's loads before working on this one
-    const int64_t tn = t + gridDim.x;
-    int gn = 0, vrows_n = 0, cc_n = 0;
-    int64_t jn = 0, r0n = 0;
-    uint4 raw_n[4];
-    if (tn < ntiles) {
-      locate(tn, gn, jn, r0n, vrows_n, cc_n);
-      fetch(r0n, vrows_n, cc_n, raw_n);
+  advance_group(pos);
+  // producer (thread 0): the next tile to load
+  Pos ppos = pos;
+  int64_t ptile = t;
+  int issued = 0, consumed = 0;
+  if (tid == 0) {
+    for (int s = 0; s < kQStages && ptile < ntiles; ++s) {
+      issue(ppos, s);
+      ++issued;
+      ptile += gridDim.x;
+      step(ppos);
     }
-    const int col = cc * kQCols + c8 * 8;
-    const bool col_ok = col < cols;
-    float v[4][8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw[i]);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v[i][k] = __bfloat162float(h[k]);
-    }
-
-    if (codes_r != nullptr) {
+  }
+  for (; t < ntiles; t += gridDim.x, ++consumed) {
+    const int s = consumed % kQStages;
+    const int g = pos.g, cc = pos.cc;
+    int64_t j, r0;
+    int vrows;
+    resolve(pos, j, r0, vrows);
+    // a stage that never lands: flag it, skip the work, leave after the
+    // end-of-tile barrier (every thread reaches it)
+    if (!mbar_wait(&full[s], static_cast<uint32_t>(consumed / kQStages) & 1u, abort_flag)) *abort_flag = 1;
+    const bool work = *abort_flag == 0;
+    uint4 raw[4];
+    {
+      const uint8_t* tile = stage_buf + s * kQTileBytes + c8 * 16;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        float a = 0.0f;
+        const int r = rbase + i;
+        raw[i] = (work && r < vrows && c8 * 16 < pitch) ? *reinterpret_cast<const uint4*>(tile + r * pitch)
+                                                       : make_uint4(0, 0, 0, 0);
+      }
+    }
+    const int col = cc * kQCols + c8 * 8;
+    const bool col_ok = work && col < cols;
+    float v[4][8];  // a bf16 is the high half of an fp32
 #pragma unroll
-        for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(v[i][k]));
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[i][2 * k] = __uint_as_float(w[k] << 16);
+        v[i][2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+    const int64_t tile_off = r0 * cols + col;  // element offset of this thread's first value
+
+    if (codes_r != nullptr) {
+      uint8_t* dst = codes_r + tile_off + static_cast<int64_t>(rbase) * cols;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float a = amax8(v[i]);
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));  // the 4 lanes of a 32-column block
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
         const int e = mx_scale_exp(a);
-        const float s = pow2_neg(e);
+        const float sc = pow2_neg(e);
         const int r = rbase + i;
         if (col_ok && r < vrows) {
-          const int64_t row = r0 + r;
-          uint2 q;
-          q.x = e4m3x4(v[i][0] * s, v[i][1] * s, v[i][2] * s, v[i][3] * s);
-          q.y = e4m3x4(v[i][4] * s, v[i][5] * s, v[i][6] * s, v[i][7] * s);
-          *reinterpret_cast<uint2*>(codes_r + row * cols + col) = q;
+          const float scv[8] = {sc, sc, sc, sc, sc, sc, sc, sc};
+          *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(v[i], scv);
           if ((c8 & 3) == 0) {
             // row-major [rows, cols/32], or the tcgen05 scale-factor atoms:
             // 512 bytes per (k-group of 4 blocks, 128 rows), row i of the
             // atom at byte (i%32)*16 + ((i/32)%4)*4 + block
-            const int64_t kb = col / 32;
-            const int64_t at = mma_layout ? ((kb >> 2) * mma_rb + (row >> 7)) * 512 + (row & 31) * 16 +
-                                                ((row >> 5) & 3) * 4 + (kb & 3)
-                                          : row * (cols / 32) + kb;
+            const int64_t row = r0 + r;
+            const int kb = col >> 5;
+            const int64_t at = mma_layout ? ((kb >> 2) * mma_rb + (row >> 7)) * 512 +
+                                                static_cast<int>(((row & 31) << 4) | (((row >> 5) & 3) << 2) | (kb & 3))
+                                          : row * (cols >> 5) + kb;
             scales_r[at] = static_cast<uint8_t>(e + 127);
           }
         }
@@ -203,29 +279,30 @@ __global__ void __launch_bounds__(kQThreads, 4)
     }
 
     if (codes_c != nullptr) {
+      float4* cm = reinterpret_cast<float4*>(&cmax[warp][c8 * 8]);
+      float c[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float a = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) a = fmaxf(a, fabsf(v[i][k]));
-        cmax[warp][c8 * 8 + k] = a;
-      }
+      for (int k = 0; k < 8; ++k)
+        c[k] = fmaxf(fmaxf(fabsf(v[0][k]), fabsf(v[1][k])), fmaxf(fabsf(v[2][k]), fabsf(v[3][k])));
+      cm[0] = make_float4(c[0], c[1], c[2], c[3]);
+      cm[1] = make_float4(c[4], c[5], c[6], c[7]);
       __syncthreads();
       {
-        float a = 0.0f;
+        float p[kQThreads / 32];
 #pragma unroll
-        for (int w = 0; w < kQThreads / 32; ++w) a = fmaxf(a, cmax[w][tid]);
+        for (int w = 0; w < kQThreads / 32; ++w) p[w] = cmax[w][tid];
+        const float a = fmaxf(fmaxf(fmaxf(p[0], p[1]), fmaxf(p[2], p[3])), fmaxf(fmaxf(p[4], p[5]), fmaxf(p[6], p[7])));
         const int e = mx_scale_exp(a);
         csf[tid] = pow2_neg(e);
         const int ccol = cc * kQCols + tid;
-        if (ccol < cols && vrows > 0) {
+        if (work && ccol < cols && vrows > 0) {
           int64_t at;
           if (mma_layout) {
             // atom (k-group of the group's blocks 4t..4t+3, 128 columns)
-            const int64_t kq = (row_offsets != nullptr ? qprefix[g] : static_cast<int64_t>(g) * qpg) + (j >> 2);
-            at = (kq * mma_cb + (ccol >> 7)) * 512 + (ccol & 31) * 16 + ((ccol >> 5) & 3) * 4 + (j & 3);
+            const int64_t kq = (ragged ? qprefix[g] : static_cast<int64_t>(g) * qpg) + (j >> 2);
+            at = (kq * mma_cb + (ccol >> 7)) * 512 + (((ccol & 31) << 4) | (((ccol >> 5) & 3) << 2) | (j & 3));
           } else {
-            at = ((row_offsets != nullptr ? bprefix[g] : static_cast<int64_t>(g) * bpg) + j) * cols + ccol;
+            at = ((ragged ? bprefix[g] : static_cast<int64_t>(g) * bpg) + j) * cols + ccol;
           }
           // offsets that overlap (only possible without a status word) must
           // not push a write past the documented allocation
@@ -233,44 +310,58 @@ __global__ void __launch_bounds__(kQThreads, 4)
         }
       }
       __syncthreads();
-      float s[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) s[k] = csf[c8 * 8 + k];
+      const float4 s0 = reinterpret_cast<const float4*>(csf)[c8 * 2];
+      const float4 s1 = reinterpret_cast<const float4*>(csf)[c8 * 2 + 1];
+      const float scc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      uint8_t* dst = codes_c + tile_off + static_cast<int64_t>(rbase) * cols;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int r = rbase + i;
-        if (col_ok && r < vrows) {
-          uint2 q;
-          q.x = e4m3x4(v[i][0] * s[0], v[i][1] * s[1], v[i][2] * s[2], v[i][3] * s[3]);
-          q.y = e4m3x4(v[i][4] * s[4], v[i][5] * s[5], v[i][6] * s[6], v[i][7] * s[7]);
-          *reinterpret_cast<uint2*>(codes_c + (r0 + r) * cols + col) = q;
+        if (col_ok && rbase + i < vrows) {
+          *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(v[i], scc);
         }
       }
-      __syncthreads();  // cmax / csf are reused by the next tile
     }
-    g = gn;
-    j = jn;
-    r0 = r0n;
-    vrows = vrows_n;
-    cc = cc_n;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) raw[i] = raw_n[i];
+    // every thread is done with stage s (and with cmax / csf): refill it
+    __syncthreads();
+    if (*abort_flag) {
+      if (tid == 0 && status != nullptr) atomicOr(status, GL_DEV_TIMEOUT);
+      break;
+    }
+    if (tid == 0 && ptile < ntiles) {
+      issue(ppos, s);
+      ++issued;
+      ptile += gridDim.x;
+      step(ppos);
+    }
+    step(pos);
+  }
+  if (tid == 0) {
+    // never leave while a load may still be writing shared memory
+    for (int k2 = consumed; k2 < issued; ++k2) mbar_wait_bounded(&full[k2 % kQStages], (k2 / kQStages) & 1);
   }
 }
 
 }  // namespace
 
 gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
-                          int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                          int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                           uint8_t* codes_c, uint8_t* scales_c, int scale_layout, cudaStream_t stream) {
-  const int smem = row_offsets != nullptr ? 2 * (G + 1) * static_cast<int>(sizeof(int64_t)) : 0;
-  if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel), smem + 16 * 1024) != cudaSuccess)
-    return GL_ERR_CUDA;
-  const int grid = num_sms() * 4;
+  // the source as a 2D bf16 tensor; box = one work unit (clamped to the tensor)
+  const uint32_t box_cols = static_cast<uint32_t>(cols < kQCols ? cols : kQCols);
+  const uint32_t box_rows = static_cast<uint32_t>(rows < kQRows ? rows : kQRows);
+  CUtensorMap tm;
+  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(cols) * 2};
+  const uint32_t box[2] = {box_cols, box_rows};
+  if (!encode_tmap(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, src, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return GL_ERR_UNSUPPORTED;
+  const int smem = 1024 + kQStages * kQTileBytes + 64 +
+                   (row_offsets != nullptr ? 2 * (G + 1) * static_cast<int>(sizeof(int64_t)) : 0);
+  if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel), smem) != cudaSuccess) return GL_ERR_CUDA;
+  const int grid = num_sms() * kQCtasPerSm;
   quantize_kernel<<<grid, kQThreads, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(src), rows, cols, row_offsets, G, status, codes_r,
-      scales_r, codes_c, scales_c,
-      static_cast<int64_t>(gl_mxfp8_scale_bytes(rows, cols, G, 1, scale_layout)),
+      tm, rows, cols, static_cast<int>(box_rows), static_cast<int>(box_cols * box_rows * 2), row_offsets, G, status,
+      codes_r, scales_r, codes_c, scales_c, static_cast<int64_t>(gl_mxfp8_scale_bytes(rows, cols, G, 1, scale_layout)),
       scale_layout == GL_SCALES_MMA ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
 }

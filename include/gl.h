@@ -186,7 +186,8 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
  *   src         device bf16 [rows, cols]
  *   row_offsets device int64[G+1] group row offsets, or NULL for G equal
  *               groups of rows/G rows (a stacked [G, rows/G, cols] weight)
- *   status      device int32 status word or NULL; non-zero -> nothing written
+ *   status      device int32 status word or NULL; non-zero -> nothing
+ *               written; a load that never lands (2 s) sets GL_DEV_TIMEOUT
  *   codes_r     NULL or device u8 [rows, cols]: rowwise codes (blocks of 32
  *               along each row)
  *   scales_r    device u8 (required with codes_r), in scale_layout:
@@ -219,7 +220,7 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
 #define GL_SCALES_ROWMAJOR 0
 #define GL_SCALES_MMA 1
 gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
-                               int G, const int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                               int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                                uint8_t* codes_c, uint8_t* scales_c, int scale_layout, void* stream);
 
 /*
