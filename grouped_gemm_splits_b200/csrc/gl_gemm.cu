@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ===================== TMA producer (both CTAs) =====================
     if (lane == 0) {
+      const uint64_t keep = l2_policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -301,14 +302,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               else    tma_load_3d(sb + c * 8192, &p.tmB, &full[stage], n0 + c * 64, kb * BK, tl.g);
             }
           } else {
+            // operand strips are read again by the neighbouring tiles of the
+            // band: keep them in L2 ahead of the streamed main_grad lines
             const int32_t row = static_cast<int32_t>(tl.r0 + kb * BK);
             const int m0 = tl.mt * C::kTileM + hr;
             const int n0 = tl.nt * C::kTileN + hb;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) tma_load_2d(sa + c * 8192, &p.tmA, &full[stage], m0 + c * 64, row);
+            for (int c = 0; c < 2; ++c) tma_load_2d_hint(sa + c * 8192, &p.tmA, &full[stage], m0 + c * 64, row, keep);
 #pragma unroll
             for (int c = 0; c < C::kBRows / 64; ++c)
-              tma_load_2d(sb + c * 8192, &p.tmB, &full[stage], n0 + c * 64, row);
+              tma_load_2d_hint(sb + c * 8192, &p.tmB, &full[stage], n0 + c * 64, row, keep);
           }
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -542,12 +545,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0 && rows_in) {
             const int kc = k0 + c * 32;
+            const uint64_t stream = l2_policy_evict_first();  // main_grad lines are touched once
             if (PG) {
-              if (p.accumulate) tma_reduce_add_2d(pg.map(tl.g), stg, kc, n0);
-              else              tma_store_2d(pg.map(tl.g), stg, kc, n0);
+              if (p.accumulate) tma_reduce_add_2d_hint(pg.map(tl.g), stg, kc, n0, stream);
+              else              tma_store_2d_hint(pg.map(tl.g), stg, kc, n0, stream);
             } else {
-              if (p.accumulate) tma_reduce_add_3d(&p.tmOut, stg, kc, n0, tl.g);
-              else              tma_store_3d(&p.tmOut, stg, kc, n0, tl.g);
+              if (p.accumulate) tma_reduce_add_3d_hint(&p.tmOut, stg, kc, n0, tl.g, stream);
+              else              tma_store_3d_hint(&p.tmOut, stg, kc, n0, tl.g, stream);
             }
             bulk_commit_group();
           }

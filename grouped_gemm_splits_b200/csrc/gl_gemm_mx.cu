@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
   if (warp == 0) {
     // ===================== TMA producer (both CTAs) =====================
     if (lane == 0) {
+      const uint64_t keep = l2_policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -362,9 +363,12 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
             const int32_t row = static_cast<int32_t>(tl.r0 + kb * BK);
             const int kq = qprefix[tl.g] + kb;  // scale k-group of this stage
             const int m0 = tl.mt * TMt + hr;
-            tma_load_2d(sa, &p.tmA, bar, m0, row);
+            // operand strips are read again by the band's neighbouring tiles:
+            // keep them in L2 ahead of the streamed main_grad lines
+            tma_load_2d_hint(sa, &p.tmA, bar, m0, row, keep);
 #pragma unroll
-            for (int c = 0; c < C::kBChunks; ++c) tma_load_2d(sb + c * 16384, &p.tmB, bar, n0 + hb + c * 128, row);
+            for (int c = 0; c < C::kBChunks; ++c)
+              tma_load_2d_hint(sb + c * 16384, &p.tmB, bar, n0 + hb + c * 128, row, keep);
             tma_load_3d(sf, &p.tmSA, bar, 0, m0 >> 7, kq);
             tma_load_3d(sf + kSfABytes, &p.tmSB, bar, 0, n0 >> 7, kq);
           }
@@ -608,12 +612,13 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
           __syncwarp();
           if (lane == 0 && rows_in) {
             const int kc = k0 + c * 32;
+            const uint64_t stream = l2_policy_evict_first();  // main_grad lines are touched once
             if (PG) {
-              if (p.accumulate) tma_reduce_add_2d(pg.map(tl.g), stg, kc, n0);
-              else              tma_store_2d(pg.map(tl.g), stg, kc, n0);
+              if (p.accumulate) tma_reduce_add_2d_hint(pg.map(tl.g), stg, kc, n0, stream);
+              else              tma_store_2d_hint(pg.map(tl.g), stg, kc, n0, stream);
             } else {
-              if (p.accumulate) tma_reduce_add_3d(&p.tmOut, stg, kc, n0, tl.g);
-              else              tma_store_3d(&p.tmOut, stg, kc, n0, tl.g);
+              if (p.accumulate) tma_reduce_add_3d_hint(&p.tmOut, stg, kc, n0, tl.g, stream);
+              else              tma_store_3d_hint(&p.tmOut, stg, kc, n0, tl.g, stream);
             }
             bulk_commit_group();
           }
