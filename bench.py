@@ -449,6 +449,23 @@ def main():
             "config": config, "status_word": status, "roofline": roof,
             "ops": ops, "gpu_launches": step.launches * args.steps, "clocks": clocks}
 
+    # Outside the step: the bias gradient (the column sums of each group's
+    # rows of dy), an HBM-bound pass over dy measured on its own.
+    db = torch.empty(step.wl.G, step.wl.N, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        gl.gl_dbias(step.dy, step.offsets, step.status, db)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(20):
+        gl.gl_dbias(step.dy, step.offsets, step.status, db)
+    e1.record()
+    torch.cuda.synchronize()
+    db_ms = e0.elapsed_time(e1) / 20
+    db_bytes = step.dy.numel() * 2 + db.numel() * 2 + (step.wl.G + 1) * 8
+    line["extras"] = {"dbias": {"ms": db_ms, "gbs": db_bytes / (db_ms / 1e3) / 1e9,
+                                "frac_of_hbm": db_bytes / (db_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                                "bytes": db_bytes, "note": "not part of the step"}}
+
     if rank == 0:
         ms_e2e, h2d, d2h, st2 = e2e_measure(step, max(3, args.steps // 2), 2)
         line["e2e"] = {"value": step.total_flops * world / (ms_e2e / 1e3) / 1e12, "unit": "TFLOP/s",

@@ -283,6 +283,17 @@ gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, co
   return gl::launch_grouped_gemm_mx(c);
 }
 
+gl_status gl_dbias(const void* dy, const int64_t* offsets, int32_t* status, int G, int64_t M, int N,
+                   gl_grouped dbias, void* stream) {
+  if (G <= 0 || G > GL_MAX_GROUPS || M < 0 || N <= 0) return GL_ERR_INVALID;
+  if ((dy == nullptr && M > 0) || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if (!grouped_ok(dbias, G)) return GL_ERR_INVALID;
+  if (N % 8 != 0) return GL_ERR_UNSUPPORTED;
+  if (M > 0 && !aligned16(dy)) return GL_ERR_UNSUPPORTED;
+  if (M == 0) dy = offsets;  // never read: every group is empty
+  return gl::launch_dbias(dy, offsets, status, G, N, dbias, to_stream(stream));
+}
+
 gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                                int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                                uint8_t* codes_c, uint8_t* scales_c, int scale_layout, void* stream) {

@@ -70,6 +70,9 @@ struct MxCall {
 
 gl_status launch_grouped_gemm_mx(const MxCall& c);
 
+gl_status launch_dbias(const void* dy, const int64_t* offsets, int32_t* status, int G, int N,
+                       gl_grouped dbias, cudaStream_t stream);
+
 gl_status launch_offsets(const int64_t* m, int G, int64_t expect_rows, int64_t out_rows,
                          int64_t* offsets, int32_t* status, cudaStream_t stream);
 

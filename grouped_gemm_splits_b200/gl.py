@@ -24,7 +24,7 @@ GL_STACKED, GL_PER_GROUP = 0, 1
 GL_SCALES_ROWMAJOR, GL_SCALES_MMA = 0, 1
 
 EXPORTED = ("gl_version", "gl_status_string", "gl_set_cta_pair", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
-            "group_quantize_mxfp8", "gl_mxfp8_scale_bytes", "gl_fwd_mxfp8", "gl_dgrad_mxfp8", "gl_wgrad_mxfp8")
+            "gl_dbias", "group_quantize_mxfp8", "gl_mxfp8_scale_bytes", "gl_fwd_mxfp8", "gl_dgrad_mxfp8", "gl_wgrad_mxfp8")
 
 
 class GlGrouped(ctypes.Structure):
@@ -62,6 +62,8 @@ def load() -> ctypes.CDLL:
     L.gl_dgrad.argtypes = [vp, GlGrouped, vp, vp, i32, i64, i32, i32, vp, i64, vp]
     L.gl_wgrad.restype = i32
     L.gl_wgrad.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, vp]
+    L.gl_dbias.restype = i32
+    L.gl_dbias.argtypes = [vp, vp, vp, i32, i64, i32, GlGrouped, vp]
     L.group_quantize_mxfp8.restype = i32
     L.group_quantize_mxfp8.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, vp, vp, i32, vp]
     L.gl_mxfp8_scale_bytes.restype = ctypes.c_size_t
@@ -184,6 +186,21 @@ def gl_wgrad(x: torch.Tensor, dy: torch.Tensor, offsets: torch.Tensor, status: t
                            M, N, K, mg, 1 if accumulate else 0, _stream()), "gl_wgrad")
     del keep
     return main_grad
+
+
+def gl_dbias(dy: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
+             dbias: Optional[TensorOrList] = None) -> TensorOrList:
+    """Bias gradient: per group, the column sums of its rows of dy (bf16 out).
+    ``dbias`` may be a [G, N] tensor or a list of G [N] tensors."""
+    G = offsets.numel() - 1
+    M, N = dy.shape
+    if dbias is None:
+        dbias = torch.empty(G, N, dtype=torch.bfloat16, device=dy.device)
+    db, keep = _grouped(dbias, G)
+    _check(load().gl_dbias(dy.data_ptr() if M > 0 else None, offsets.data_ptr(), status.data_ptr(), G, M, N, db,
+                           _stream()), "gl_dbias")
+    del keep
+    return dbias
 
 
 def mxfp8_scale_bytes(rows: int, cols: int, G: int, colwise: bool, mma: bool) -> int:

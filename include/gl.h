@@ -170,6 +170,21 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
                    int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream);
 
 /*
+ * gl_dbias -- bias gradient: db_i[n] = sum of dy[r, n] over the rows r of
+ * group i (``grouped_linear.py`` ops/basic fuser_backward: with a bias, each
+ * split of grad_output is summed over its rows).  fp32 accumulation, one
+ * round-to-nearest-even to bf16 per output; an empty group gets zeros.
+ *
+ *   dy       device bf16 [M, N] (rows packed by group)
+ *   offsets  device int64[G+1] from gl_offsets
+ *   status   device int32 status word (required); non-zero -> nothing written
+ *   dbias    bf16 [G, N] stacked or G pointers to [N]; every element written
+ * Limits: N % 8 == 0; dy 16-byte aligned.  Asynchronous on `stream`.
+ */
+gl_status gl_dbias(const void* dy, const int64_t* offsets, int32_t* status, int G, int64_t M, int N,
+                   gl_grouped dbias, void* stream);
+
+/*
  * group_quantize_mxfp8 -- MXFP8 (E4M3 codes, E8M0 block scales) cast of a
  * bf16 [rows, cols] tensor whose rows form G groups.
  *

@@ -58,7 +58,12 @@ def test_host_side_validation_without_gpu():
     assert lib.group_quantize_mxfp8(16, 8, 48, None, 1, None, 16, 16, None, None, 0, None) == gl.GL_ERR_UNSUPPORTED
     assert lib.group_quantize_mxfp8(16, 8, 64, None, 1, None, None, None, None, None, 0, None) == gl.GL_ERR_INVALID
     assert lib.group_quantize_mxfp8(16, 9, 64, None, 2, None, 16, 16, None, None, 0, None) == gl.GL_ERR_INVALID
-    # k-group-major scales need cols % 128 == 0; unknown layout codes are rejected
+    # dbias: G <= 0, null status, N % 8 != 0
+    st = gl.GlGrouped(gl.GL_STACKED, 16, None)
+    assert lib.gl_dbias(16, 16, 16, 0, 8, 8, st, None) == gl.GL_ERR_INVALID
+    assert lib.gl_dbias(16, 16, None, 2, 8, 8, st, None) == gl.GL_ERR_INVALID
+    assert lib.gl_dbias(16, 16, 16, 2, 8, 12, st, None) == gl.GL_ERR_UNSUPPORTED
+    # MMA-layout scales need cols % 128 == 0; unknown layout codes are rejected
     assert lib.group_quantize_mxfp8(16, 8, 96, None, 1, None, 16, 16, None, None, 1, None) == gl.GL_ERR_UNSUPPORTED
     assert lib.group_quantize_mxfp8(16, 8, 128, None, 1, None, 16, 16, None, None, 7, None) == gl.GL_ERR_INVALID
 
