@@ -233,20 +233,24 @@ def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] 
         G = row_offsets.numel() - 1
     dev = src.device
     out = {} if out is None else out
+    def need(key, make):
+        if key not in out:  # allocate only what the caller did not supply
+            out[key] = make()
+
     if rowwise:
-        out.setdefault("codes_r", torch.empty(rows, cols, dtype=torch.uint8, device=dev))
+        need("codes_r", lambda: torch.empty(rows, cols, dtype=torch.uint8, device=dev))
         if mma_scales:
-            out.setdefault("scales_r", torch.empty(mxfp8_scale_bytes(rows, cols, G, False, True),
-                                                   dtype=torch.uint8, device=dev))
+            need("scales_r", lambda: torch.empty(mxfp8_scale_bytes(rows, cols, G, False, True), dtype=torch.uint8,
+                                                 device=dev))
         else:
-            out.setdefault("scales_r", torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev))
+            need("scales_r", lambda: torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev))
     if colwise:
-        out.setdefault("codes_c", torch.empty(rows, cols, dtype=torch.uint8, device=dev))
+        need("codes_c", lambda: torch.empty(rows, cols, dtype=torch.uint8, device=dev))
         if mma_scales:
-            out.setdefault("scales_c", torch.empty(mxfp8_scale_bytes(rows, cols, G, True, True),
-                                                   dtype=torch.uint8, device=dev))
+            need("scales_c", lambda: torch.empty(mxfp8_scale_bytes(rows, cols, G, True, True), dtype=torch.uint8,
+                                                 device=dev))
         else:
-            out.setdefault("scales_c", torch.empty((rows + 31) // 32 + G, cols, dtype=torch.uint8, device=dev))
+            need("scales_c", lambda: torch.empty((rows + 31) // 32 + G, cols, dtype=torch.uint8, device=dev))
     _check(load().group_quantize_mxfp8(
         src2.data_ptr(), rows, cols, _ptr(row_offsets), G, _ptr(status),
         _ptr(out.get("codes_r")) if rowwise else None, _ptr(out.get("scales_r")) if rowwise else None,

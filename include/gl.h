@@ -202,7 +202,9 @@ gl_status gl_dbias(const void* dy, const int64_t* offsets, int32_t* status, int 
  *   row_offsets device int64[G+1] group row offsets, or NULL for G equal
  *               groups of rows/G rows (a stacked [G, rows/G, cols] weight)
  *   status      device int32 status word or NULL; non-zero -> nothing
- *               written; a load that never lands (2 s) sets GL_DEV_TIMEOUT
+ *               written (so a flag set on the device makes a captured weight
+ *               cast a no-op on CUDA-graph replays); a load that never lands
+ *               (2 s) sets GL_DEV_TIMEOUT
  *   codes_r     NULL or device u8 [rows, cols]: rowwise codes (blocks of 32
  *               along each row)
  *   scales_r    device u8 (required with codes_r), in scale_layout:
