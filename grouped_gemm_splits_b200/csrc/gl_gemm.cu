@@ -38,7 +38,6 @@ namespace gl {
 namespace {
 
 constexpr int BK = 64;  // contraction elements per stage (one 128-byte swizzle row)
-constexpr int kThreads = 192;
 constexpr int kPG = 64;  // per-group tensor maps carried by one launch
 constexpr int kSmemBudget = 196608;
 constexpr int kBand = 8;  // tile rows per rasterisation band
@@ -51,7 +50,11 @@ struct Cfg {
   static constexpr int kABytes = 128 * BK * 2;     // 16 KB
   static constexpr int kBBytes = kBRows * BK * 2;  // 32 KB (CG 1) or 16 KB (CG 2)
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStagingBytes = (MODE == kWgrad) ? 2 * 128 * 32 * 4 : 0;  // 2 x 16 KB
+  // epilogue warps, one per TMEM lane quarter (eight for wgrad measured no
+  // faster and cost a pipeline stage of staging space)
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kStagingBytes = (MODE == kWgrad) ? kEpiWarps * 32 * 32 * 4 : 0;  // one 4 KB transpose per epilogue warp
   static constexpr int kStages = (kSmemBudget - kStagingBytes) / kStageBytes;
   static constexpr int kBarOffset = kStages * kStageBytes + kStagingBytes;
   static constexpr int kBarBytes = 256;
@@ -61,18 +64,20 @@ struct Cfg {
   static constexpr int kBMN = (MODE == kFwd) ? 0 : 1;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, kTileN, kAMN, kBMN);
   static_assert(kStages >= 3, "pipeline too shallow");
+  // dynamic shared memory at the largest group count (tile prefix), + alignment slack
+  static_assert(kBarOffset + kBarBytes + (GL_MAX_GROUPS + 1) * 4 + 1024 <= 232448, "shared memory");
   static_assert(kBarOffset % 1024 == 0, "stage alignment");
 };
 
 struct GemmParams {
   CUtensorMap tmA;    // FWD x{K,M} box{64,128}; DGRAD dy{N,M} box{64,128}; WGRAD dy{N,M} box{64,64}
   CUtensorMap tmB;    // stacked W{K,N,G}: FWD box{64,BRows,1}, DGRAD box{64,64,1}; WGRAD x{K,M} box{64,64}
-  CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,32,1}
   const int64_t* offsets;  // G+1 entries
   int32_t* status;
   int64_t M;
   int64_t out_rows;
   void* out;                  // FWD y / DGRAD dx (bf16)
+  float* mg;                  // WGRAD stacked main_grad [G, N, K]
   const __nv_bfloat16* bias;  // stacked bias [G,N] or null
   int G;
   int N, K;
@@ -82,16 +87,19 @@ struct GemmParams {
 
 template <bool PG>
 struct PGArgs {
-  CUtensorMap tm[kPG];  // FWD/DGRAD: W_g{K,N}; WGRAD: main_grad_g{K,N}
+  CUtensorMap tm[kPG];  // FWD/DGRAD: W_g{K,N}
   const __nv_bfloat16* bias[kPG];
+  float* mg[kPG];       // WGRAD: main_grad_g [N, K]
   __device__ const CUtensorMap* map(int g) const { return &tm[g]; }
   __device__ const __nv_bfloat16* b(int g) const { return bias[g]; }
+  __device__ float* m(int g) const { return mg[g]; }
 };
 template <>
 struct PGArgs<false> {
   int unused;
   __device__ const CUtensorMap* map(int) const { return nullptr; }
   __device__ const __nv_bfloat16* b(int) const { return nullptr; }
+  __device__ float* m(int) const { return nullptr; }
 };
 
 struct Tile {
@@ -134,8 +142,16 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const Gemm
   const int base_mt = band * kBand;
   const int bh = min(kBand, mtg - base_mt);
   const int within = local - band * kBand * ntg;
-  tl.mt = base_mt + within % bh;
-  tl.nt = within / bh;
+  if (MODE == kWgrad) {
+    // row-major inside the band: consecutive tiles cover the same 256 main_grad
+    // rows across the whole K width, so the fp32 read-modify-write of the
+    // tiles in flight reaches DRAM as long contiguous runs
+    tl.mt = base_mt + within / ntg;
+    tl.nt = within % ntg;
+  } else {
+    tl.mt = base_mt + within % bh;
+    tl.nt = within / bh;
+  }
   if (MODE == kWgrad) {
     tl.r0 = o0;
     tl.r1 = o0 + m;
@@ -181,7 +197,7 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* sa, uint8_t* sb, int r_f
 }
 
 template <int MODE, int CG, bool PG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ PGArgs<PG> pg) {
   using C = Cfg<MODE, CG>;
   extern __shared__ uint8_t smem_raw[];
@@ -210,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4 * CG);  // one arrival per epilogue warp of the pair
+      mbar_init(&tempty[b], C::kEpiWarps * CG);  // one arrival per epilogue warp of the pair
     }
     mbar_init(mma_done, 1);
     fence_barrier_init();
@@ -264,7 +280,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
     if (!PG || MODE == kWgrad) tma_prefetch_desc(&p.tmB);
-    if (MODE == kWgrad && !PG) tma_prefetch_desc(&p.tmOut);
   }
   tc_fence_before();
   __syncthreads();
@@ -447,7 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_leader = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : 0u;
     int it = 0;
-    int chunk_ctr = 0;
     for (int t = pair; t < total; t += npairs, ++it) {
       const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
       const int buf = it & 1;
@@ -512,21 +526,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // main_grad rows n0.. (this warp's 32 TMEM lanes) x cols k0 + 32c: each
-        // epilogue warp stages and stores its own [32 x 32] fp32 boxes
-        float* wstage = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes) + (warp - 2) * (2 * 32 * 32);
+        // main_grad rows n0 + 0..31 (this warp's TMEM lanes) x columns k0 + 32c..:
+        // each [32 x 32] fp32 chunk goes through a 4 KB per-warp shared-memory
+        // transpose (16-byte pieces, XOR-swizzled: conflict-free both ways), so
+        // that 8 lanes cover one row's 128 contiguous bytes, then leaves as
+        // coalesced 16-byte vector reductions (accumulate) or stores
+        // (overwrite): full-line transactions, many in flight, no waits.
+        float* stg = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes) + (warp - 2) * (32 * 32);
+        constexpr int kCols = C::kTileN / (C::kEpiWarps / 4);  // columns of this warp (its half)
+        const int half = (warp - 2) >> 2;
         const int n0 = tl.mt * C::kTileM + hr + q * 32;
-        const int k0 = tl.nt * C::kTileN;
-        const int nchunks = min(C::kTileN / 32, ceil_div_i(p.K - k0, 32));
+        const int k0 = tl.nt * C::kTileN + half * kCols;
+        const int nchunks = max(0, min(kCols / 32, ceil_div_i(p.K - k0, 32)));
         const bool have_acc = tl.num_kb > 0;
-        const bool rows_in = n0 < p.N;  // the pair's second half may lie past N
-        for (int c = 0; c < nchunks; ++c, ++chunk_ctr) {
-          float* stg = wstage + (chunk_ctr & 1) * (32 * 32);
-          if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
-          __syncwarp();
+        float* gbase = PG ? pg.m(tl.g) : p.mg + static_cast<int64_t>(tl.g) * p.N * p.K;
+        const int sub = lane >> 3, piece = lane & 7;  // read side: row 4i + sub, 16-byte piece
+        for (int c = 0; c < nchunks; ++c) {
           uint32_t r[32];
           if (have_acc) {
-            tmem_ld_32x32b_x32(tacc + c * 32, r);
+            tmem_ld_32x32b_x32(tacc + half * kCols + c * 32, r);
             tmem_ld_wait();
             tmem_reg_fence(r);
           } else {
@@ -534,31 +552,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) r[j] = 0u;
           }
           if (c == nchunks - 1) release_acc();
-          // row `lane` of a [32 x 32] fp32 box, 128-byte swizzle
-          uint8_t* rowp = reinterpret_cast<uint8_t*>(stg) + lane * 128;
+          float* mine = stg + lane * 32;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int pj = j ^ (lane & 7);
-            *reinterpret_cast<uint4*>(rowp + pj * 16) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-          }
-          fence_proxy_async_smem();
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(mine + ((j ^ (lane & 7)) << 2)) =
+                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
           __syncwarp();
-          if (lane == 0 && rows_in) {
-            const int kc = k0 + c * 32;
-            const uint64_t stream = l2_policy_evict_first();  // main_grad lines are touched once
-            if (PG) {
-              if (p.accumulate) tma_reduce_add_2d_hint(pg.map(tl.g), stg, kc, n0, stream);
-              else              tma_store_2d_hint(pg.map(tl.g), stg, kc, n0, stream);
-            } else {
-              if (p.accumulate) tma_reduce_add_3d_hint(&p.tmOut, stg, kc, n0, tl.g, stream);
-              else              tma_store_3d_hint(&p.tmOut, stg, kc, n0, tl.g, stream);
+          const int col = k0 + c * 32 + piece * 4;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int row = 4 * i + sub;
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + row * 32 + ((piece ^ (row & 7)) << 2));
+            if (n0 + row < p.N && col < p.K) {  // K % 8 == 0: four columns are all in or all out
+              float* dst = gbase + static_cast<int64_t>(n0 + row) * p.K + col;
+              if (p.accumulate) red_add_v4(dst, v.x, v.y, v.z, v.w);
+              else *reinterpret_cast<uint4*>(dst) = v;
             }
-            bulk_commit_group();
           }
+          __syncwarp();  // the next chunk overwrites the transpose buffer
         }
+        if (nchunks == 0) release_acc();  // this warp's half lies past K: nothing to read
       }
     }
-    if (MODE == kWgrad && lane == 0) bulk_wait_group<0>();  // stores of this warp done
   }
 
   tc_fence_before();
@@ -591,10 +606,10 @@ bool make_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uin
   return encode_tmap(m, dt, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-cudaLaunchConfig_t pair_config(int grid, int smem, cudaStream_t stream, cudaLaunchAttribute* attr) {
+cudaLaunchConfig_t pair_config(int grid, int threads, int smem, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -608,7 +623,7 @@ cudaLaunchConfig_t pair_config(int grid, int smem, cudaStream_t stream, cudaLaun
 
 // Persistent grid: one CTA per SM, or as many CTA pairs as can be resident.
 template <typename Kern>
-int grid_for(Kern kern, int cg, int smem) {
+int grid_for(Kern kern, int cg, int threads, int smem) {
   if (cg == 1) return num_sms();
   static std::mutex mu;
   static std::unordered_map<const void*, int> cache;
@@ -621,7 +636,7 @@ int grid_for(Kern kern, int cg, int smem) {
     if (it != cache.end()) return it->second;
   }
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config(2 * (num_sms() / 2), smem, nullptr, attr);
+  cudaLaunchConfig_t cfg = pair_config(2 * (num_sms() / 2), threads, smem, nullptr, attr);
   int nclusters = 0;
   if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters <= 0)
     nclusters = num_sms() / 2;
@@ -636,12 +651,13 @@ gl_status launch_one(const GemmParams& prm, const PGArgs<PG>& pga, int G, cudaSt
   const int smem = smem_bytes_for<MODE, CG>(G);
   auto kern = grouped_gemm_kernel<MODE, CG, PG>;
   if (set_max_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return GL_ERR_CUDA;
-  const int grid = grid_for(kern, CG, smem);
+  constexpr int threads = Cfg<MODE, CG>::kThreads;
+  const int grid = grid_for(kern, CG, threads, smem);
   if (CG == 1) {
-    kern<<<grid, kThreads, smem, stream>>>(prm, pga);
+    kern<<<grid, threads, smem, stream>>>(prm, pga);
   } else {
     cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = pair_config(grid, smem, stream, attr);
+    cudaLaunchConfig_t cfg = pair_config(grid, threads, smem, stream, attr);
     if (cudaLaunchKernelEx(&cfg, kern, prm, pga) != cudaSuccess) return GL_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
@@ -678,8 +694,7 @@ gl_status launch_mode(const GemmCall& c) {
   if (stacked && (!prm.has_bias || bias_stacked)) {
     if (MODE == kFwd) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, BK, Cf::kBRows, BF, 2);
     if (MODE == kDgrad) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, 64, BK, BF, 2);
-    if (MODE == kWgrad)
-      ok &= make_3d(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+    if (MODE == kWgrad) prm.mg = static_cast<float*>(const_cast<void*>(c.out_grouped.base));
     if (!ok) return GL_ERR_UNSUPPORTED;
     prm.offsets = c.offsets;
     prm.G = c.G;
@@ -710,7 +725,7 @@ gl_status launch_mode(const GemmCall& c) {
         const void* gp = (c.out_grouped.mode == GL_STACKED)
                              ? static_cast<const uint8_t*>(c.out_grouped.base) + static_cast<size_t>(g) * c.N * c.K * 4
                              : c.out_grouped.ptrs[g];
-        ok &= make_2d(&pga->tm[i], gp, c.K, c.N, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+        pga->mg[i] = static_cast<float*>(const_cast<void*>(gp));
       }
     }
     if (!ok) { st = GL_ERR_UNSUPPORTED; break; }

@@ -13,8 +13,10 @@
 // fprop / dgrad: TN = 256 and one fp32 accumulator (256 TMEM columns); eight
 // epilogue warps copy it to registers and free it at once, so the next tile's
 // MMAs overlap the stores.  wgrad: TN = 192 and two accumulators (384
-// columns); four epilogue warps stage fp32 boxes for TMA reduce-adds.  The
-// remaining TMEM columns hold the scale-factor slots.
+// columns); eight epilogue warps (half the columns each) transpose 32 x 32
+// fp32 chunks through shared memory and add them into main_grad with
+// coalesced 16-byte vector reductions.  The remaining TMEM columns hold the
+// scale-factor slots.
 //
 // Per stage (128 contraction elements = four MMAs of K=32) the producer
 // TMA-loads the codes (128-byte swizzle) and the scales.  The scales arrive
@@ -61,7 +63,7 @@ template <int MODE, int CG>
 struct CfgMX {
   static constexpr int kTN = (MODE == kWgrad) ? 192 : 256;  // accumulator columns
   static constexpr int kAccBufs = (MODE == kWgrad) ? 2 : 1;
-  static constexpr int kEpiWarps = (MODE == kWgrad) ? 4 : 8;
+  static constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, half the columns each
   static constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, 1 MMA / relay, then epilogue
   static constexpr int kSfCol0 = kAccBufs * kTN;        // first TMEM column of the scale-factor slots
   static constexpr int kTileM = 128 * CG;
@@ -74,15 +76,17 @@ struct CfgMX {
   static_assert((kTN % 128 == 0 ? 0 : 64) + kTN <= 128 * kAtomsB && kTN % 64 == 0,
                 "B tile must stay inside the loaded scale atoms");
   static constexpr int kStageBytes = kABytes + kBAlloc + kSfBytes;  // 50 KB (CG 1) / 34 KB (CG 2)
-  static constexpr int kStagingBytes = (MODE == kWgrad) ? 4 * 2 * 32 * 32 * 4 : 0;
+  static constexpr int kStagingBytes = (MODE == kWgrad) ? kEpiWarps * 32 * 32 * 4 : 0;  // one 4 KB transpose per epilogue warp
   static constexpr int kStages = CG == 2 ? ((MODE == kWgrad) ? 5 : 6) : ((MODE == kWgrad) ? 3 : 4);
   static constexpr int kTx = kABytes + kBLoad + kSfABytes + kAtomsB * 512;
   static constexpr int kStagingOffset = kStages * kStageBytes;
-  static constexpr int kBarOffset = (kStagingOffset + kStagingBytes + 1023) / 1024 * 1024;
+  static constexpr int kBarOffset = kStagingOffset + kStagingBytes;
   static constexpr int kPrefixOffset = kBarOffset + 256;
   static_assert((2 * kStages + 5) * 8 + 16 <= 256, "barrier area");
   static_assert(kSfCol0 + kSfSlots * kSfSlotCols <= 512, "TMEM columns");
-  static_assert(kStageBytes % 1024 == 0 && kStagingOffset % 1024 == 0, "alignment");
+  // dynamic shared memory at the largest group count (tile and scale prefixes), + alignment slack
+  static_assert(kPrefixOffset + 2 * (GL_MAX_GROUPS_MXFP8 + 1) * 4 + 1024 <= 232448, "shared memory");
+  static_assert(kStageBytes % 1024 == 0, "alignment");
   // operand majorness in shared memory (1 = MN-major)
   static constexpr int kAMN = (MODE == kWgrad) ? 1 : 0;
   static constexpr int kBMN = (MODE == kFwd) ? 0 : 1;
@@ -93,12 +97,12 @@ struct MxParams {
   CUtensorMap tmB;    // stacked B codes: FWD W{K,N,G} box{128,BRows,1}; DGRAD Wc{K,N,G} box{128,128,1}; WGRAD x_c{K,M} box{128,128}
   CUtensorMap tmSA;   // A scale atoms (u32 {128, atoms, k-groups}) box{128,1,1}
   CUtensorMap tmSB;   // stacked B scale atoms box{128,2,1}
-  CUtensorMap tmOut;  // WGRAD stacked main_grad{K,N,G} box{32,32,1}
   const int64_t* offsets;      // this launch's G+1 offsets
   const int64_t* offsets_all;  // every group's offsets (WGRAD scale k-groups of earlier groups)
   int32_t* status;
   int64_t out_rows;
   void* out;
+  float* mg;  // WGRAD stacked main_grad [G, N, K]
   const __nv_bfloat16* bias;
   int G;
   int g0;  // index of this launch's first group
@@ -109,12 +113,14 @@ struct MxParams {
 
 template <bool PG>
 struct MxPG {
-  CUtensorMap tm[kPG];   // FWD/DGRAD: B codes of group g; WGRAD: main_grad of group g
+  CUtensorMap tm[kPG];   // FWD/DGRAD: B codes of group g
   CUtensorMap tms[kPG];  // FWD/DGRAD: B scale atoms of group g
   const __nv_bfloat16* bias[kPG];
+  float* mg[kPG];        // WGRAD: main_grad of group g [N, K]
   __device__ const CUtensorMap* map(int g) const { return &tm[g]; }
   __device__ const CUtensorMap* smap(int g) const { return &tms[g]; }
   __device__ const __nv_bfloat16* b(int g) const { return bias[g]; }
+  __device__ float* m(int g) const { return mg[g]; }
 };
 template <>
 struct MxPG<false> {
@@ -122,6 +128,7 @@ struct MxPG<false> {
   __device__ const CUtensorMap* map(int) const { return nullptr; }
   __device__ const CUtensorMap* smap(int) const { return nullptr; }
   __device__ const __nv_bfloat16* b(int) const { return nullptr; }
+  __device__ float* m(int) const { return nullptr; }
 };
 
 struct Tile {
@@ -165,8 +172,16 @@ __device__ __forceinline__ Tile decode(int t, const int* prefix, const MxParams&
   const int base_mt = band * kBand;
   const int bh = min(kBand, mtg - base_mt);
   const int within = local - band * kBand * ntg;
-  tl.mt = base_mt + within % bh;
-  tl.nt = within / bh;
+  if (MODE == kWgrad) {
+    // row-major inside the band: consecutive tiles cover the same 256 main_grad
+    // rows across the whole K width, so the fp32 read-modify-write of the
+    // tiles in flight reaches DRAM as long contiguous runs
+    tl.mt = base_mt + within / ntg;
+    tl.nt = within % ntg;
+  } else {
+    tl.mt = base_mt + within % bh;
+    tl.nt = within / bh;
+  }
   tl.rlo = o0;
   tl.r1 = o0 + m;
   if (MODE == kWgrad) {
@@ -516,7 +531,6 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_leader = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : 0u;
     int it = 0;
-    int chunk_ctr = 0;
     for (int t = pair; t < total; t += npairs, ++it) {
       const Tile tl = decode<MODE, CG>(t, prefix, p);
       const int buf = it % C::kAccBufs;
@@ -580,21 +594,24 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
           }
         }
       } else {
-        // main_grad rows n0.. (this warp's 32 TMEM lanes) x cols k0 + 32c: each
-        // epilogue warp stages and stores its own [32 x 32] fp32 boxes
-        float* wstage = reinterpret_cast<float*>(smem + C::kStagingOffset) + (warp - 2) * (2 * 32 * 32);
+        // main_grad rows n0 + 0..31 (this warp's TMEM lanes) x columns k0 + 32c..:
+        // each [32 x 32] fp32 chunk goes through a 4 KB per-warp shared-memory
+        // transpose (16-byte pieces, XOR-swizzled: conflict-free both ways), so
+        // that 8 lanes cover one row's 128 contiguous bytes, then leaves as
+        // coalesced 16-byte vector reductions (accumulate) or stores
+        // (overwrite): full-line transactions, many in flight, no waits.
+        float* stg = reinterpret_cast<float*>(smem + C::kStagingOffset) + (warp - 2) * (32 * 32);
+        constexpr int kCols = TN / 2;  // columns of this warp (its half)
         const int n0 = tl.mt * TMt + hr + q * 32;
-        const int k0 = tl.nt * TN;
-        const int nchunks = min(TN / 32, cdiv(p.K - k0, 32));
+        const int k0 = tl.nt * TN + h * kCols;
+        const int nchunks = max(0, min(kCols / 32, cdiv(p.K - k0, 32)));
         const bool have_acc = tl.num_kb > 0;
-        const bool rows_in = n0 < p.N;
-        for (int c = 0; c < nchunks; ++c, ++chunk_ctr) {
-          float* stg = wstage + (chunk_ctr & 1) * (32 * 32);
-          if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
-          __syncwarp();
+        float* gbase = PG ? pg.m(tl.g) : p.mg + static_cast<int64_t>(tl.g) * p.N * p.K;
+        const int sub = lane >> 3, piece = lane & 7;  // read side: row 4i + sub, 16-byte piece
+        for (int c = 0; c < nchunks; ++c) {
           uint32_t r[32];
           if (have_acc) {
-            tmem_ld_32x32b_x32(tacc + c * 32, r);
+            tmem_ld_32x32b_x32(tacc + h * kCols + c * 32, r);
             tmem_ld_wait();
             tmem_reg_fence(r);
           } else {
@@ -602,30 +619,28 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
             for (int j = 0; j < 32; ++j) r[j] = 0u;
           }
           if (c == nchunks - 1) release_acc();
-          uint8_t* rowp = reinterpret_cast<uint8_t*>(stg) + lane * 128;
+          float* mine = stg + lane * 32;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int pj = j ^ (lane & 7);
-            *reinterpret_cast<uint4*>(rowp + pj * 16) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-          }
-          fence_proxy_async_smem();
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(mine + ((j ^ (lane & 7)) << 2)) =
+                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
           __syncwarp();
-          if (lane == 0 && rows_in) {
-            const int kc = k0 + c * 32;
-            const uint64_t stream = l2_policy_evict_first();  // main_grad lines are touched once
-            if (PG) {
-              if (p.accumulate) tma_reduce_add_2d_hint(pg.map(tl.g), stg, kc, n0, stream);
-              else              tma_store_2d_hint(pg.map(tl.g), stg, kc, n0, stream);
-            } else {
-              if (p.accumulate) tma_reduce_add_3d_hint(&p.tmOut, stg, kc, n0, tl.g, stream);
-              else              tma_store_3d_hint(&p.tmOut, stg, kc, n0, tl.g, stream);
+          const int col = k0 + c * 32 + piece * 4;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int row = 4 * i + sub;
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + row * 32 + ((piece ^ (row & 7)) << 2));
+            if (n0 + row < p.N && col < p.K) {  // K % 128 == 0: four columns are all in or all out
+              float* dst = gbase + static_cast<int64_t>(n0 + row) * p.K + col;
+              if (p.accumulate) red_add_v4(dst, v.x, v.y, v.z, v.w);
+              else *reinterpret_cast<uint4*>(dst) = v;
             }
-            bulk_commit_group();
           }
+          __syncwarp();  // the next chunk overwrites the transpose buffer
         }
+        if (nchunks == 0) release_acc();  // this warp's half lies past K: nothing to read
       }
     }
-    if (MODE == kWgrad && lane == 0) bulk_wait_group<0>();  // stores of this warp done
   }
 
   tc_fence_before();
@@ -774,7 +789,7 @@ gl_status mx_mode(const MxCall& c) {
       ok &= map3(&prm.tmB, c.w.base, c.K, c.N, c.G, 1, 128, 128, U8);
       ok &= map_atoms(&prm.tmSB, c.ws.base, KA, G * NA, KA, kAtomsB);  // G groups of N/128 k-groups
     } else {
-      ok &= map3(&prm.tmOut, c.out_grouped.base, c.K, c.N, c.G, 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+      prm.mg = static_cast<float*>(const_cast<void*>(c.out_grouped.base));
     }
     if (!ok) return GL_ERR_UNSUPPORTED;
     prm.offsets = c.offsets;
@@ -792,9 +807,8 @@ gl_status mx_mode(const MxCall& c) {
     for (int i = 0; i < cg; ++i) {
       const int g = g0 + i;
       if (MODE == kWgrad) {
-        const void* gp = group_ptr(c.out_grouped, g, static_cast<size_t>(c.N) * c.K * 4);
-        ok &= map2(&pga->tm[i], gp, c.K, c.N, static_cast<uint64_t>(c.K) * 4, 32, 32,
-                   CU_TENSOR_MAP_DATA_TYPE_FLOAT32, SW);
+        pga->mg[i] = static_cast<float*>(
+            const_cast<void*>(group_ptr(c.out_grouped, g, static_cast<size_t>(c.N) * c.K * 4)));
         continue;
       }
       const void* wp = group_ptr(c.w, g, static_cast<size_t>(c.N) * c.K);
