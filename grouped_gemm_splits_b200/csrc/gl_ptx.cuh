@@ -122,6 +122,8 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, ui
       : "memory");
 }
 
+// L2 cache policy for TMA loads of operand strips that neighbouring tiles
+// read again: evict_last, ahead of the streamed fp32 main_grad lines.
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -137,8 +139,8 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* t
       : "memory");
 }
 
-// fp32 main_grad update of four consecutive values (16-byte aligned):
-// a vector reduction performed in L2 (accumulate) or a plain vector store.
+// Add four consecutive fp32 values (16-byte aligned) into global memory: one
+// vector reduction, performed in L2.
 __device__ __forceinline__ void red_add_v4(float* dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(__uint_as_float(a)),
                "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
