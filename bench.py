@@ -314,16 +314,36 @@ def oracle_sample(workload: str = WORKLOAD, seed_offset: int = 0, rows_per_group
 
 
 # ----------------------------------------------------------------------------
-def dist_setup(gpus: int):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+def rank_env():
+    """(world size, rank, local rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_setup(world: int, local: int) -> None:
+    """One process per GPU: a NCCL process group (short timeout) when N > 1.
+    The path has no exchange step, so the group only carries the barrier and
+    the max-over-ranks reduction of the timed region."""
     if world > 1:
         import datetime
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
-    return world, rank, local
+
+
+def max_over_ranks(ms: float, device) -> float:
+    """The job's time for a timed region: the slowest rank's (an all-reduce
+    MAX over the process group); the value itself on a single process."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank_step: float, world: int, ms_step: float) -> float:
+    """Whole-job throughput: every replica's flops over the slowest rank's time."""
+    return flops_per_rank_step * world / (ms_step / 1e3) / 1e12
 
 
 def main():
@@ -336,7 +356,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = rank_env()
     wl = synth.WORKLOADS[args.workload]
     config = {"workload": f"{args.workload}: G={wl.G} K={wl.K} N={wl.N} rows={wl.rows}"
                           f"{' (output buffers ' + str(wl.out_rows) + ' rows)' if wl.out_rows > wl.rows else ''}, "
@@ -370,6 +390,7 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
+    dist_setup(world, local)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     gl.load()
@@ -395,11 +416,7 @@ def main():
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
-    ms_total = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
     ms_step = ms_total / args.steps
     status = int(step.status.item()) | int(step.mx.status.item())
 
@@ -441,7 +458,7 @@ def main():
                 "unit": "GB/s", "frac": ops[dom]["gbs"] / pk["hbm_gbs"],
                 "peak_source": f"{pk['source']} copy bandwidth",
                 "traffic": MEASURED_TRAFFIC.get(args.workload, {}).get(dom)}
-    value = step.total_flops * world / (ms_step / 1e3) / 1e12
+    value = job_tflops(step.total_flops, world, ms_step)
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
@@ -466,10 +483,14 @@ def main():
                                 "frac_of_hbm": db_bytes / (db_ms / 1e3) / 1e9 / pk["hbm_gbs"],
                                 "bytes": db_bytes, "note": "not part of the step"}}
 
+    # end to end on every rank (host buffers in, status out), slowest rank's time
+    if world > 1:
+        torch.distributed.barrier()
+    ms_e2e, h2d, d2h, st2 = e2e_measure(step, max(3, args.steps // 2), 2)
+    ms_e2e = max_over_ranks(ms_e2e, dev)
+    line["e2e"] = {"value": job_tflops(step.total_flops, world, ms_e2e), "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
     if rank == 0:
-        ms_e2e, h2d, d2h, st2 = e2e_measure(step, max(3, args.steps // 2), 2)
-        line["e2e"] = {"value": step.total_flops * world / (ms_e2e / 1e3) / 1e12, "unit": "TFLOP/s",
-                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
         if world == 1 and not args.no_cpu_baseline:
             fl, sec, thr, desc = oracle_sample(args.workload)
             line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOP/s", "cores": thr,
