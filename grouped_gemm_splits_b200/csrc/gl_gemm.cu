@@ -19,8 +19,9 @@
 // Roles: warp 0 TMA producer (128-byte swizzled boxes into a ring of
 // shared-memory stages), warp 1 TMEM owner and MMA issuer (leader) or stage
 // relay (peer), warps 2-5 epilogue (TMEM -> registers; bias + bf16 rounding
-// and row-clipped stores for FWD/DGRAD; TMA reduce-add or TMA store of fp32
-// main_grad boxes for WGRAD).  Two accumulators in TMEM let a tile's
+// and row-clipped stores for FWD/DGRAD; for WGRAD 32 x 32 fp32 chunks
+// transposed through shared memory and added into main_grad with coalesced
+// 16-byte vector reductions, or stored).  Two accumulators in TMEM let a tile's
 // epilogue overlap the next tile's main loop.  Tiles are enumerated group by
 // group from the device offsets (tile prefix in shared memory): empty groups
 // cost nothing and the host never learns the split sizes.
