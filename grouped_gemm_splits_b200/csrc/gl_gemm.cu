@@ -40,7 +40,7 @@ namespace {
 
 constexpr int BK = 64;  // contraction elements per stage (one 128-byte swizzle row)
 constexpr int kPG = 64;  // per-group tensor maps carried by one launch
-constexpr int kSmemBudget = 196608;
+constexpr int kSmemBudget = 212992;  // 6 stages of 32 KB + (wgrad) 16 KB of epilogue transposes
 constexpr int kBand = 8;  // tile rows per rasterisation band
 
 template <int MODE, int CG>
