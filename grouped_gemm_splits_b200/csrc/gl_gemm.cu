@@ -462,11 +462,28 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_leader = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : 0u;
+    auto prefetch_mg = [&](const Tile& tn) {
+      constexpr int kCols = C::kTileN / (C::kEpiWarps / 4);
+      const int n = tn.mt * C::kTileM + hr + q * 32 + lane;
+      const int k0 = tn.nt * C::kTileN + ((warp - 2) >> 2) * kCols;
+      const int cols = min(kCols, p.K - k0);
+      if (n < p.N && cols > 0) {
+        const float* gb = PG ? pg.m(tn.g) : p.mg + static_cast<int64_t>(tn.g) * p.N * p.K;
+        l2_prefetch_bulk(gb + static_cast<int64_t>(n) * p.K + k0, static_cast<uint32_t>(cols) * 4u);
+      }
+    };
     int it = 0;
     for (int t = pair; t < total; t += npairs, ++it) {
       const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
       const int buf = it & 1;
       const uint32_t tph = (it >> 1) & 1;
+      if (MODE == kWgrad && p.accumulate) {
+        // while the tile's main loop runs, pull this lane's main_grad row
+        // segment into L2 with one bulk request, so that the reductions below
+        // find their lines there (prefetching one tile further ahead measured
+        // slower on small groups)
+        prefetch_mg(tl);
+      }
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
       if (!ok) report_abort(abort_flag, p.status);
       if (!ok) break;

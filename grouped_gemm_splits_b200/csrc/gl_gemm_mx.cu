@@ -530,11 +530,27 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
     const int h = (warp - 2) >> 2;         // FWD/DGRAD: 128-column half of the tile
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_leader = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : 0u;
+    auto prefetch_mg = [&](const Tile& tn) {
+      const int n = tn.mt * TMt + hr + q * 32 + lane;
+      const int k0 = tn.nt * TN + h * (TN / 2);
+      const int cols = min(TN / 2, p.K - k0);
+      if (n < p.N && cols > 0) {
+        const float* gb = PG ? pg.m(tn.g) : p.mg + static_cast<int64_t>(tn.g) * p.N * p.K;
+        l2_prefetch_bulk(gb + static_cast<int64_t>(n) * p.K + k0, static_cast<uint32_t>(cols) * 4u);
+      }
+    };
     int it = 0;
     for (int t = pair; t < total; t += npairs, ++it) {
       const Tile tl = decode<MODE, CG>(t, prefix, p);
       const int buf = it % C::kAccBufs;
       const uint32_t tph = (it / C::kAccBufs) & 1;
+      if (MODE == kWgrad && p.accumulate) {
+        // while the tile's main loop runs, pull this lane's main_grad row
+        // segment into L2 with one bulk request, so that the reductions below
+        // find their lines there (prefetching one tile further ahead measured
+        // slower on small groups)
+        prefetch_mg(tl);
+      }
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
       if (!ok) report_abort(abort_flag, p.status);
       if (!ok) break;

@@ -139,6 +139,13 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* t
       : "memory");
 }
 
+// Hint: bring [src, src + bytes) into L2 with one bulk request (no completion
+// to wait for).  src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
+
 // Add four consecutive fp32 values (16-byte aligned) into global memory: one
 // vector reduction, performed in L2.
 __device__ __forceinline__ void red_add_v4(float* dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
