@@ -252,28 +252,36 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
 
     if (codes_r != nullptr) {
       uint8_t* dst = codes_r + tile_off + static_cast<int64_t>(rbase) * cols;
+      uint32_t ebytes = 0;  // biased scale exponents of this thread's 4 rows, row i in byte i
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float a = amax8(v[i]);
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));  // the 4 lanes of a 32-column block
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
         const int e = mx_scale_exp(a);
+        ebytes |= static_cast<uint32_t>(e + 127) << (8 * i);
         const float sc = pow2_neg(e);
-        const int r = rbase + i;
-        if (col_ok && r < vrows) {
+        if (col_ok && rbase + i < vrows) {
           const float scv[8] = {sc, sc, sc, sc, sc, sc, sc, sc};
           *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(v[i], scv);
-          if ((c8 & 3) == 0) {
-            // row-major [rows, cols/32], or the tcgen05 scale-factor atoms:
-            // 512 bytes per (k-group of 4 blocks, 128 rows), row i of the
-            // atom at byte (i%32)*16 + ((i/32)%4)*4 + block
-            const int64_t row = r0 + r;
-            const int kb = col >> 5;
-            const int64_t at = mma_layout ? ((kb >> 2) * mma_rb + (row >> 7)) * 512 +
-                                                static_cast<int>(((row & 31) << 4) | (((row >> 5) & 3) << 2) | (kb & 3))
-                                          : row * (cols >> 5) + kb;
-            scales_r[at] = static_cast<uint8_t>(e + 127);
-          }
+        }
+      }
+      // the warp's 4 rows x 8 blocks of 32 columns are 32 scales: lane L
+      // writes the one of row L/8, block L%8 (taken from that block's first
+      // lane), so every lane stores one byte instead of a quarter storing four
+      {
+        const int ri = lane >> 3, blk = lane & 7;
+        const uint32_t eb = __shfl_sync(0xffffffffu, ebytes, blk * 4);
+        const int kb = (cc * kQCols >> 5) + blk;
+        if (work && (kb << 5) < cols && rbase + ri < vrows) {
+          // row-major [rows, cols/32], or the tcgen05 scale-factor atoms:
+          // 512 bytes per (k-group of 4 blocks, 128 rows), row i of the
+          // atom at byte (i%32)*16 + ((i/32)%4)*4 + block
+          const int64_t row = r0 + rbase + ri;
+          const int64_t at = mma_layout ? ((kb >> 2) * mma_rb + (row >> 7)) * 512 +
+                                              static_cast<int>(((row & 31) << 4) | (((row >> 5) & 3) << 2) | (kb & 3))
+                                        : row * (cols >> 5) + kb;
+          scales_r[at] = static_cast<uint8_t>(eb >> (8 * ri));
         }
       }
     }
