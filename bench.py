@@ -40,7 +40,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # entry must be removed when its kernel changes.
 MEASURED_TRAFFIC = {
     "bf16_g8": {"fwd": 2463018752, "dgrad": 3406094848,
-                "quant_x": 220894464, "quant_w": 1878619648, "quant_dy": 910224896,
                 "fwd_mx": 1204673536, "dgrad_mx": 1414253568},
 }
 
