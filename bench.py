@@ -499,6 +499,35 @@ def main():
                                 "frac_of_hbm": db_bytes / (db_ms / 1e3) / 1e9 / pk["hbm_gbs"],
                                 "bytes": db_bytes, "note": "not part of the step"}}
 
+    # Also outside the step: the cast of dy fused with its bias gradient (one
+    # pass over dy; group_quantize_mxfp8_dbias) on the MXFP8 half's splits,
+    # against that half's cast of dy plus gl_dbias on the same splits.
+    mx = step.mx
+
+    def timed(f, n=20):
+        for _ in range(3):
+            f()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(n):
+            f()
+        a1.record()
+        torch.cuda.synchronize()
+        return a0.elapsed_time(a1) / n
+
+    ws = torch.empty(gl.dbias_workspace_bytes(mx.wl.rows, mx.wl.N, mx.wl.G), dtype=torch.uint8, device=dev)
+    qd, dbm = {}, torch.empty(mx.wl.G, mx.wl.N, dtype=torch.bfloat16, device=dev)
+    fused_ms = timed(lambda: gl.group_quantize_mxfp8_dbias(mx.dy, mx.offsets, mx.status, out=qd, mma_scales=True,
+                                                           dbias=dbm, workspace=ws))
+    sep_db_ms = timed(lambda: gl.gl_dbias(mx.dy, mx.offsets, mx.status, dbm))
+    cd_bytes = mx.bytes["quant_dy"] + dbm.numel() * 2
+    line["extras"]["cast_dbias"] = {
+        "ms": fused_ms, "gbs": cd_bytes / (fused_ms / 1e3) / 1e9,
+        "frac_of_hbm": cd_bytes / (fused_ms / 1e3) / 1e9 / pk["hbm_gbs"], "bytes": cd_bytes,
+        "separate_ms": ops["quant_dy"]["ms"] + sep_db_ms,
+        "note": "MXFP8 cast of dy (rowwise + columnwise) with its bias gradient in one pass; separate_ms = the "
+                "step's cast of dy + gl_dbias on the same splits; not part of the step"}
+
     # end to end on every rank (host buffers in, status out), slowest rank's time
     if world > 1:
         torch.distributed.barrier()

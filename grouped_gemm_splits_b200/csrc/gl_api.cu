@@ -294,12 +294,16 @@ gl_status gl_dbias(const void* dy, const int64_t* offsets, int32_t* status, int 
   return gl::launch_dbias(dy, offsets, status, G, N, dbias, to_stream(stream));
 }
 
-gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
-                               int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
-                               uint8_t* codes_c, uint8_t* scales_c, int scale_layout, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Argument checks shared by the two cast entry points (GL_OK when valid).
+gl_status check_quantize_args(const void* src, int64_t rows, int cols, const int64_t* row_offsets, int G,
+                              const uint8_t* codes_r, const uint8_t* scales_r, const uint8_t* codes_c,
+                              const uint8_t* scales_c, int scale_layout) {
   if (src == nullptr || rows < 0 || cols <= 0 || G <= 0 || G > GL_MAX_GROUPS) return GL_ERR_INVALID;
   if (codes_r == nullptr && codes_c == nullptr) return GL_ERR_INVALID;
-  if ((codes_r != nullptr) != (scales_r != nullptr) && codes_r != nullptr) return GL_ERR_INVALID;
   if (codes_r != nullptr && scales_r == nullptr) return GL_ERR_INVALID;
   if (codes_c != nullptr && scales_c == nullptr) return GL_ERR_INVALID;
   if (cols % 32 != 0) return GL_ERR_UNSUPPORTED;
@@ -310,9 +314,54 @@ gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const in
   if (!aligned16(src) || (codes_r && (reinterpret_cast<uintptr_t>(codes_r) & 7u)) ||
       (codes_c && (reinterpret_cast<uintptr_t>(codes_c) & 7u)))
     return GL_ERR_UNSUPPORTED;
+  return GL_OK;
+}
+
+// Workspace of the fused cast + bias gradient: the groups' first blocks
+// (int64[G+1], padded to 256 bytes), then the per-block column sums.
+size_t dbias_ws_head(int G) { return ((static_cast<size_t>(G) + 1) * 8 + 255) / 256 * 256; }
+int64_t dbias_ws_blocks(int64_t rows, int G) { return (rows + 31) / 32 + G; }
+
+}  // namespace
+
+extern "C" {
+
+gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
+                               int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                               uint8_t* codes_c, uint8_t* scales_c, int scale_layout, void* stream) {
+  const gl_status st =
+      check_quantize_args(src, rows, cols, row_offsets, G, codes_r, scales_r, codes_c, scales_c, scale_layout);
+  if (st != GL_OK) return st;
   if (rows == 0) return GL_OK;
-  return gl::launch_quantize(src, rows, cols, row_offsets, G, status, codes_r, scales_r, codes_c,
-                             scales_c, scale_layout, to_stream(stream));
+  return gl::launch_quantize(src, rows, cols, row_offsets, G, status, codes_r, scales_r, codes_c, scales_c,
+                             scale_layout, nullptr, 0, nullptr, to_stream(stream));
+}
+
+size_t gl_dbias_workspace_bytes(int64_t rows, int cols, int G) {
+  if (rows < 0 || cols <= 0 || G <= 0) return 0;
+  return dbias_ws_head(G) + static_cast<size_t>(dbias_ws_blocks(rows, G)) * static_cast<size_t>(cols) * 4;
+}
+
+gl_status group_quantize_mxfp8_dbias(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
+                                     int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                                     uint8_t* codes_c, uint8_t* scales_c, int scale_layout, gl_grouped dbias,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  const gl_status st =
+      check_quantize_args(src, rows, cols, row_offsets, G, codes_r, scales_r, codes_c, scales_c, scale_layout);
+  if (st != GL_OK) return st;
+  if (row_offsets == nullptr || status == nullptr || workspace == nullptr) return GL_ERR_INVALID;
+  if (!grouped_ok(dbias, G)) return GL_ERR_INVALID;
+  if (workspace_bytes < gl_dbias_workspace_bytes(rows, cols, G)) return GL_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GL_ERR_UNSUPPORTED;
+  cudaStream_t s = to_stream(stream);
+  if (rows == 0)  // every group is empty: zeros (the source is never read)
+    return gl::launch_dbias(row_offsets, row_offsets, status, G, cols, dbias, s);
+  int64_t* prefix = static_cast<int64_t*>(workspace);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dbias_ws_head(G));
+  const gl_status q = gl::launch_quantize(src, rows, cols, row_offsets, G, status, codes_r, scales_r, codes_c,
+                                          scales_c, scale_layout, part, dbias_ws_blocks(rows, G), prefix, s);
+  if (q != GL_OK) return q;
+  return gl::launch_dbias_partials(part, prefix, status, G, cols, dbias, s);
 }
 
 size_t gl_mxfp8_scale_bytes(int64_t rows, int cols, int G, int colwise, int scale_layout) {

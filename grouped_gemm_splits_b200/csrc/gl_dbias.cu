@@ -14,6 +14,11 @@
 // and rounds to bf16.  Splitting every group 8 ways keeps the largest group
 // of a skewed split from serialising the pass.  HBM-bound: dy is read once;
 // the output is [G, N].  An empty group gets zeros.
+//
+// The same kernel, on fp32 input, finishes the bias gradient that the MXFP8
+// cast of dy computes on the way (gl_quantize.cu): its rows are then the
+// cast's per-32-row-block column sums and the group offsets count blocks.
+// Every level adds in a fixed order, so the result is deterministic.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -36,8 +41,17 @@ struct DbiasPG {
   __nv_bfloat16* ptr[kDPG];
 };
 
+// four consecutive columns of one row as fp32
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+  return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                     __uint_as_float(v.y & 0xFFFF0000u));
+}
+__device__ __forceinline__ float4 load4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+
+template <typename T>
 __global__ void __cluster_dims__(kDCluster, 1, 1) __launch_bounds__(kDThreads)
-    dbias_kernel(const __nv_bfloat16* __restrict__ dy, const int64_t* __restrict__ offsets,
+    dbias_kernel(const T* __restrict__ dy, const int64_t* __restrict__ offsets,
                  const int32_t* __restrict__ status, int N, int strips, __nv_bfloat16* __restrict__ out,
                  const __grid_constant__ DbiasPG pg, int per_group) {
   __shared__ __align__(16) float part[kDWarps][kDCols];
@@ -54,28 +68,27 @@ __global__ void __cluster_dims__(kDCluster, 1, 1) __launch_bounds__(kDThreads)
 
   float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (col_ok) {
-    const __nv_bfloat16* base = dy + col;
+    const T* base = dy + col;
     int64_t r = r0 + static_cast<int>(crank) * kDWarps + warp;
     // kDUnroll independent rows per iteration keep loads in flight
     for (; r + (kDUnroll - 1) * kStride < r1; r += kDUnroll * kStride) {
-      uint2 v[kDUnroll];
+      float4 v[kDUnroll];
 #pragma unroll
-      for (int u = 0; u < kDUnroll; ++u)
-        v[u] = __ldg(reinterpret_cast<const uint2*>(base + (r + u * kStride) * N));
+      for (int u = 0; u < kDUnroll; ++u) v[u] = load4(base + (r + u * kStride) * N);
 #pragma unroll
       for (int u = 0; u < kDUnroll; ++u) {
-        acc[0] += __uint_as_float(v[u].x << 16);
-        acc[1] += __uint_as_float(v[u].x & 0xFFFF0000u);
-        acc[2] += __uint_as_float(v[u].y << 16);
-        acc[3] += __uint_as_float(v[u].y & 0xFFFF0000u);
+        acc[0] += v[u].x;
+        acc[1] += v[u].y;
+        acc[2] += v[u].z;
+        acc[3] += v[u].w;
       }
     }
     for (; r < r1; r += kStride) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(base + r * N));
-      acc[0] += __uint_as_float(v.x << 16);
-      acc[1] += __uint_as_float(v.x & 0xFFFF0000u);
-      acc[2] += __uint_as_float(v.y << 16);
-      acc[3] += __uint_as_float(v.y & 0xFFFF0000u);
+      const float4 v = load4(base + r * N);
+      acc[0] += v.x;
+      acc[1] += v.y;
+      acc[2] += v.z;
+      acc[3] += v.w;
     }
   }
   *reinterpret_cast<float4*>(&part[warp][lane * 4]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -105,17 +118,15 @@ __global__ void __cluster_dims__(kDCluster, 1, 1) __launch_bounds__(kDThreads)
   cluster_sync();  // the first CTA has read every peer's shared memory
 }
 
-}  // namespace
-
-gl_status launch_dbias(const void* dy, const int64_t* offsets, int32_t* status, int G, int N,
-                       gl_grouped dbias, cudaStream_t stream) {
+template <typename T>
+gl_status launch_segmented_colsum(const T* src, const int64_t* offsets, int32_t* status, int G, int N,
+                                  gl_grouped dbias, cudaStream_t stream) {
   const int strips = (N + kDCols - 1) / kDCols;
-  const auto* d = static_cast<const __nv_bfloat16*>(dy);
   if (dbias.mode == GL_STACKED) {
     DbiasPG none;
     memset(&none, 0, sizeof(none));
-    dbias_kernel<<<G * strips * kDCluster, kDThreads, 0, stream>>>(d, offsets, status, N, strips,
-                                                       static_cast<__nv_bfloat16*>(const_cast<void*>(dbias.base)), none, 0);
+    dbias_kernel<T><<<G * strips * kDCluster, kDThreads, 0, stream>>>(
+        src, offsets, status, N, strips, static_cast<__nv_bfloat16*>(const_cast<void*>(dbias.base)), none, 0);
     return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
   }
   DbiasPG pg;
@@ -123,10 +134,23 @@ gl_status launch_dbias(const void* dy, const int64_t* offsets, int32_t* status, 
     const int cg = std::min(kDPG, G - g0);
     memset(&pg, 0, sizeof(pg));
     for (int i = 0; i < cg; ++i) pg.ptr[i] = static_cast<__nv_bfloat16*>(const_cast<void*>(dbias.ptrs[g0 + i]));
-    dbias_kernel<<<cg * strips * kDCluster, kDThreads, 0, stream>>>(d, offsets + g0, status, N, strips, nullptr, pg, 1);
+    dbias_kernel<T><<<cg * strips * kDCluster, kDThreads, 0, stream>>>(src, offsets + g0, status, N, strips, nullptr,
+                                                                       pg, 1);
     if (cudaGetLastError() != cudaSuccess) return GL_ERR_CUDA;
   }
   return GL_OK;
+}
+
+}  // namespace
+
+gl_status launch_dbias(const void* dy, const int64_t* offsets, int32_t* status, int G, int N,
+                       gl_grouped dbias, cudaStream_t stream) {
+  return launch_segmented_colsum(static_cast<const __nv_bfloat16*>(dy), offsets, status, G, N, dbias, stream);
+}
+
+gl_status launch_dbias_partials(const float* part, const int64_t* part_prefix, int32_t* status, int G, int N,
+                                gl_grouped dbias, cudaStream_t stream) {
+  return launch_segmented_colsum(part, part_prefix, status, G, N, dbias, stream);
 }
 
 }  // namespace gl

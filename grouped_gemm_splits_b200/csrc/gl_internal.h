@@ -76,8 +76,18 @@ gl_status launch_dbias(const void* dy, const int64_t* offsets, int32_t* status, 
 gl_status launch_offsets(const int64_t* m, int G, int64_t expect_rows, int64_t out_rows,
                          int64_t* offsets, int32_t* status, cudaStream_t stream);
 
+// part != NULL: also the per-(32-row block, column) fp32 sums of the source
+// (part [part_blocks, cols]) and the groups' first blocks (part_prefix
+// int64[G+1]); row_offsets required.
 gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                           int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
-                          uint8_t* codes_c, uint8_t* scales_c, int scale_layout, cudaStream_t stream);
+                          uint8_t* codes_c, uint8_t* scales_c, int scale_layout, float* part,
+                          int64_t part_blocks, int64_t* part_prefix, cudaStream_t stream);
+
+// Bias gradient from the cast's partials: dbias_g[n] = sum over the blocks
+// [part_prefix[g], part_prefix[g+1]) of part[b, n], in block order, rounded
+// once to bf16.
+gl_status launch_dbias_partials(const float* part, const int64_t* part_prefix, int32_t* status, int G, int N,
+                                gl_grouped dbias, cudaStream_t stream);
 
 }  // namespace gl

@@ -17,6 +17,14 @@
 // CTA first builds the per-group block prefixes in shared memory.
 // Memory-bound: 2 bytes read and up to 2 bytes (+1/16 for scales) written per
 // element.
+//
+// With a bias gradient (the cast of dy; fuser_backward sums each split of
+// grad_output over its rows next to quantizing it), the same pass also adds
+// every work unit's 32 rows per column in fp32 -- a thread its 4 rows, then
+// the 8 warps in order through shared memory -- and stores one fp32 partial
+// per (32-row block, column) in a caller workspace; dbias_partials_kernel
+// (gl_dbias.cu) adds each group's partials in block order.  The sums are
+// deterministic: no atomics, a fixed order at every level.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -83,12 +91,17 @@ __device__ __forceinline__ float amax8(const float (&v)[8]) {
   return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
 
+// kDbias: also write the per-block column sums (part: [part_blocks, cols]
+// fp32, block b of the launch in row b; part_prefix: the groups' first
+// blocks, int64[G+1], written by CTA 0).
+template <bool kDbias>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_src, int64_t rows, int cols, int box_rows,
                     int tile_bytes, const int64_t* __restrict__ row_offsets, int G, int32_t* status,
                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r,
                     uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, int64_t scales_c_bytes,
-                    int mma_layout) {
+                    int mma_layout, float* __restrict__ part, int64_t part_blocks,
+                    int64_t* __restrict__ part_prefix) {
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* qsmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_buf = qsmem;                                                  // kQStages x 16 KB
@@ -98,6 +111,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   int64_t* qprefix = bprefix + G + 1;                                                  // G+1 (ragged)
   __shared__ __align__(16) float cmax[kQThreads / 32][kQCols];  // per-warp column maxima
   __shared__ __align__(16) float csf[kQCols];                     // 2^-e of each column
+  __shared__ __align__(16) float csum[kDbias ? kQThreads / 32 : 1][kQCols];  // per-warp column sums
   if (status != nullptr && *reinterpret_cast<volatile int32_t*>(status) != 0) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
@@ -134,6 +148,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     if (lane == 0) { bprefix[0] = 0; qprefix[0] = 0; }
   }
   __syncthreads();
+  if (kDbias && blockIdx.x == 0 && row_offsets != nullptr)
+    for (int i = tid; i <= G; i += kQThreads) part_prefix[i] = bprefix[i];
   const int64_t nblocks = (row_offsets != nullptr) ? bprefix[G] : bpg * G;
   const int ncc = (cols + kQCols - 1) / kQCols;
   const int64_t ntiles = nblocks * ncc;
@@ -286,6 +302,25 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       }
     }
 
+    // bias gradient: this thread's 4 rows per column (rows past the block's
+    // valid rows were loaded as zeros), published with the next barrier
+    if (kDbias) {
+      float cs[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) cs[k] = ((v[0][k] + v[1][k]) + v[2][k]) + v[3][k];
+      float4* cp = reinterpret_cast<float4*>(&csum[warp][c8 * 8]);
+      cp[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
+      cp[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
+    }
+    // thread tid: column cc*256 + tid of this block, the 8 warps in order
+    auto store_partial = [&]() {
+      float a = csum[0][tid];
+#pragma unroll
+      for (int w = 1; w < kQThreads / 32; ++w) a += csum[w][tid];
+      const int ccol = cc * kQCols + tid;
+      if (work && ccol < cols && pos.rb < part_blocks) part[pos.rb * cols + ccol] = a;
+    };
+
     if (codes_c != nullptr) {
       float4* cm = reinterpret_cast<float4*>(&cmax[warp][c8 * 8]);
       float c[8];
@@ -317,6 +352,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
           if (at < scales_c_bytes) scales_c[at] = static_cast<uint8_t>(e + 127);
         }
       }
+      if (kDbias) store_partial();  // csum complete since the barrier above
       __syncthreads();
       const float4 s0 = reinterpret_cast<const float4*>(csf)[c8 * 2];
       const float4 s1 = reinterpret_cast<const float4*>(csf)[c8 * 2 + 1];
@@ -329,7 +365,11 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         }
       }
     }
-    // every thread is done with stage s (and with cmax / csf): refill it
+    if (kDbias && codes_c == nullptr) {
+      __syncthreads();  // csum complete
+      store_partial();
+    }
+    // every thread is done with stage s (and with cmax / csf / csum): refill it
     __syncthreads();
     if (*abort_flag) {
       if (tid == 0 && status != nullptr) atomicOr(status, GL_DEV_TIMEOUT);
@@ -353,7 +393,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
 
 gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
                           int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
-                          uint8_t* codes_c, uint8_t* scales_c, int scale_layout, cudaStream_t stream) {
+                          uint8_t* codes_c, uint8_t* scales_c, int scale_layout, float* part,
+                          int64_t part_blocks, int64_t* part_prefix, cudaStream_t stream) {
   // the source as a 2D bf16 tensor; box = one work unit (clamped to the tensor)
   const uint32_t box_cols = static_cast<uint32_t>(cols < kQCols ? cols : kQCols);
   const uint32_t box_rows = static_cast<uint32_t>(rows < kQRows ? rows : kQRows);
@@ -365,12 +406,21 @@ gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t
     return GL_ERR_UNSUPPORTED;
   const int smem = 1024 + kQStages * kQTileBytes + 64 +
                    (row_offsets != nullptr ? 2 * (G + 1) * static_cast<int>(sizeof(int64_t)) : 0);
-  if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel), smem) != cudaSuccess) return GL_ERR_CUDA;
   const int grid = num_sms() * kQCtasPerSm;
-  quantize_kernel<<<grid, kQThreads, smem, stream>>>(
-      tm, rows, cols, static_cast<int>(box_rows), static_cast<int>(box_cols * box_rows * 2), row_offsets, G, status,
-      codes_r, scales_r, codes_c, scales_c, static_cast<int64_t>(gl_mxfp8_scale_bytes(rows, cols, G, 1, scale_layout)),
-      scale_layout == GL_SCALES_MMA ? 1 : 0);
+  const int tile_bytes = static_cast<int>(box_cols * box_rows * 2);
+  const int64_t sc_bytes = static_cast<int64_t>(gl_mxfp8_scale_bytes(rows, cols, G, 1, scale_layout));
+  const int mma = scale_layout == GL_SCALES_MMA ? 1 : 0;
+  if (part != nullptr) {
+    if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel<true>), smem) != cudaSuccess) return GL_ERR_CUDA;
+    quantize_kernel<true><<<grid, kQThreads, smem, stream>>>(
+        tm, rows, cols, static_cast<int>(box_rows), tile_bytes, row_offsets, G, status, codes_r, scales_r, codes_c,
+        scales_c, sc_bytes, mma, part, part_blocks, part_prefix);
+  } else {
+    if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel<false>), smem) != cudaSuccess) return GL_ERR_CUDA;
+    quantize_kernel<false><<<grid, kQThreads, smem, stream>>>(
+        tm, rows, cols, static_cast<int>(box_rows), tile_bytes, row_offsets, G, status, codes_r, scales_r, codes_c,
+        scales_c, sc_bytes, mma, nullptr, 0, nullptr);
+  }
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
 }
 

@@ -24,7 +24,8 @@ GL_STACKED, GL_PER_GROUP = 0, 1
 GL_SCALES_ROWMAJOR, GL_SCALES_MMA = 0, 1
 
 EXPORTED = ("gl_version", "gl_status_string", "gl_set_cta_pair", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
-            "gl_dbias", "group_quantize_mxfp8", "gl_mxfp8_scale_bytes", "gl_fwd_mxfp8", "gl_dgrad_mxfp8", "gl_wgrad_mxfp8")
+            "gl_dbias", "group_quantize_mxfp8", "gl_mxfp8_scale_bytes", "gl_dbias_workspace_bytes",
+            "group_quantize_mxfp8_dbias", "gl_fwd_mxfp8", "gl_dgrad_mxfp8", "gl_wgrad_mxfp8")
 
 
 class GlGrouped(ctypes.Structure):
@@ -68,6 +69,11 @@ def load() -> ctypes.CDLL:
     L.group_quantize_mxfp8.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, vp, vp, i32, vp]
     L.gl_mxfp8_scale_bytes.restype = ctypes.c_size_t
     L.gl_mxfp8_scale_bytes.argtypes = [i64, i32, i32, i32, i32]
+    L.gl_dbias_workspace_bytes.restype = ctypes.c_size_t
+    L.gl_dbias_workspace_bytes.argtypes = [i64, i32, i32]
+    L.group_quantize_mxfp8_dbias.restype = i32
+    L.group_quantize_mxfp8_dbias.argtypes = [vp, i64, i32, vp, i32, vp, vp, vp, vp, vp, i32, GlGrouped, vp,
+                                             ctypes.c_size_t, vp]
     L.gl_fwd_mxfp8.restype = i32
     L.gl_fwd_mxfp8.argtypes = [vp, vp, GlGrouped, GlGrouped, ctypes.POINTER(GlGrouped), vp, vp, i32, i64, i32,
                                i32, vp, i64, vp]
@@ -223,16 +229,34 @@ def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] 
     ``mma_scales`` flat byte arrays in the tcgen05 scale-factor layout that the
     MXFP8 GEMMs read (``GL_SCALES_MMA``).
     """
+    src2, rows, cols, G = _cast_shape(src, row_offsets, G)
+    out = _cast_outputs(src2, G, rowwise, colwise, out, mma_scales)
+    _check(load().group_quantize_mxfp8(
+        src2.data_ptr(), rows, cols, _ptr(row_offsets), G, _ptr(status),
+        _ptr(out.get("codes_r")) if rowwise else None, _ptr(out.get("scales_r")) if rowwise else None,
+        _ptr(out.get("codes_c")) if colwise else None, _ptr(out.get("scales_c")) if colwise else None,
+        GL_SCALES_MMA if mma_scales else GL_SCALES_ROWMAJOR, _stream()), "group_quantize_mxfp8")
+    return out
+
+
+def _cast_shape(src: torch.Tensor, row_offsets: Optional[torch.Tensor], G: int):
     if src.dim() == 3:
         G = src.shape[0]
         src2 = src.reshape(-1, src.shape[-1])
     else:
         src2 = src
-    rows, cols = src2.shape
     if row_offsets is not None:
         G = row_offsets.numel() - 1
-    dev = src.device
+    rows, cols = src2.shape
+    return src2, rows, cols, G
+
+
+def _cast_outputs(src2: torch.Tensor, G: int, rowwise: bool, colwise: bool, out: Optional[dict],
+                  mma_scales: bool) -> dict:
+    rows, cols = src2.shape
+    dev = src2.device
     out = {} if out is None else out
+
     def need(key, make):
         if key not in out:  # allocate only what the caller did not supply
             out[key] = make()
@@ -251,12 +275,42 @@ def group_quantize_mxfp8(src: torch.Tensor, row_offsets: Optional[torch.Tensor] 
                                                  device=dev))
         else:
             need("scales_c", lambda: torch.empty((rows + 31) // 32 + G, cols, dtype=torch.uint8, device=dev))
-    _check(load().group_quantize_mxfp8(
-        src2.data_ptr(), rows, cols, _ptr(row_offsets), G, _ptr(status),
+    return out
+
+
+def dbias_workspace_bytes(rows: int, cols: int, G: int) -> int:
+    """Workspace bytes of :func:`group_quantize_mxfp8_dbias` (``gl_dbias_workspace_bytes``)."""
+    n = load().gl_dbias_workspace_bytes(rows, cols, G)
+    if n == 0:
+        raise GlError(f"gl_dbias_workspace_bytes: invalid arguments ({rows}, {cols}, {G})")
+    return n
+
+
+def group_quantize_mxfp8_dbias(dy: torch.Tensor, row_offsets: torch.Tensor, status: torch.Tensor,
+                               rowwise: bool = True, colwise: bool = True, out: Optional[dict] = None,
+                               mma_scales: bool = False, dbias: Optional[TensorOrList] = None,
+                               workspace: Optional[torch.Tensor] = None):
+    """:func:`group_quantize_mxfp8` of a ragged dy that also returns its bias
+    gradient (per group, the column sums of its rows; bf16 [G, cols] or a list
+    of G [cols] tensors) from the same pass.  ``workspace`` (uint8, at least
+    :func:`dbias_workspace_bytes`, 256-byte aligned) is allocated when absent.
+    Returns (codes/scales dict, dbias)."""
+    src2, rows, cols, G = _cast_shape(dy, row_offsets, 1)
+    out = _cast_outputs(src2, G, rowwise, colwise, out, mma_scales)
+    if dbias is None:
+        dbias = torch.empty(G, cols, dtype=torch.bfloat16, device=dy.device)
+    nbytes = dbias_workspace_bytes(rows, cols, G)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dy.device)
+    db, keep = _grouped(dbias, G)
+    _check(load().group_quantize_mxfp8_dbias(
+        src2.data_ptr(), rows, cols, row_offsets.data_ptr(), G, status.data_ptr(),
         _ptr(out.get("codes_r")) if rowwise else None, _ptr(out.get("scales_r")) if rowwise else None,
         _ptr(out.get("codes_c")) if colwise else None, _ptr(out.get("scales_c")) if colwise else None,
-        GL_SCALES_MMA if mma_scales else GL_SCALES_ROWMAJOR, _stream()), "group_quantize_mxfp8")
-    return out
+        GL_SCALES_MMA if mma_scales else GL_SCALES_ROWMAJOR, db, workspace.data_ptr(), workspace.numel(),
+        _stream()), "group_quantize_mxfp8_dbias")
+    del keep
+    return out, dbias
 
 
 # ---------------------------------------------------------------- MXFP8 GEMMs

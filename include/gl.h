@@ -250,6 +250,47 @@ gl_status group_quantize_mxfp8(const void* src, int64_t rows, int cols, const in
 size_t gl_mxfp8_scale_bytes(int64_t rows, int cols, int G, int colwise, int scale_layout);
 
 /*
+ * group_quantize_mxfp8_dbias -- group_quantize_mxfp8 of a ragged bf16 dy
+ * that also writes its bias gradient from the same read of dy:
+ * db_i[n] = sum of dy[r, n] over the rows r of group i (``grouped_linear.py``
+ * ops/basic fuser_backward with MXFP8 quantizers: grad_output is quantized per
+ * split and, with a bias, each split is summed over its rows; doing both in
+ * one pass saves a full read of dy).
+ *
+ * Each 32-row block of a group adds its rows per column in fp32 in a fixed
+ * order and stores one fp32 partial per (block, column) in the workspace; a
+ * second kernel adds each group's partials in a fixed order and rounds once
+ * to bf16 (round-to-nearest-even).  The result is deterministic; it agrees
+ * with gl_dbias to fp32 rounding (the two add in different orders).  An
+ * empty group gets zeros.
+ *
+ *   src .. scale_layout   as for group_quantize_mxfp8; row_offsets required
+ *   status      device int32 status word (required); non-zero -> nothing
+ *               written
+ *   dbias       bf16 [G, cols] stacked or G pointers to [cols]; every element
+ *               written
+ *   workspace   device scratch of workspace_bytes >= gl_dbias_workspace_bytes
+ *               (rows, cols, G), 256-byte aligned, owned by the caller; its
+ *               contents on entry do not matter and it may be reused once the
+ *               call's work on `stream` has finished
+ * Errors: GL_ERR_INVALID for a NULL row_offsets / status / workspace or a
+ * workspace that is too small; GL_ERR_UNSUPPORTED for a misaligned
+ * workspace; otherwise those of group_quantize_mxfp8.  Asynchronous on
+ * `stream` (two launches).
+ */
+gl_status group_quantize_mxfp8_dbias(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
+                                     int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                                     uint8_t* codes_c, uint8_t* scales_c, int scale_layout, gl_grouped dbias,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * gl_dbias_workspace_bytes -- workspace bytes for group_quantize_mxfp8_dbias:
+ * int64[G+1] block offsets (padded to 256 bytes) + fp32
+ * [ceil(rows/32) + G, cols] partials.  Host-only; 0 for invalid arguments.
+ */
+size_t gl_dbias_workspace_bytes(int64_t rows, int cols, int G);
+
+/*
  * MXFP8 grouped GEMMs -- the three products of gl_fwd / gl_dgrad / gl_wgrad
  * on MXFP8 operands (E4M3 codes, E8M0 scale per 32 contraction elements, as
  * written by group_quantize_mxfp8), computed as

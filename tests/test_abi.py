@@ -68,6 +68,31 @@ def test_host_side_validation_without_gpu():
     assert lib.group_quantize_mxfp8(16, 8, 128, None, 1, None, 16, 16, None, None, 7, None) == gl.GL_ERR_INVALID
 
 
+def test_fused_cast_dbias_validation_and_workspace_size():
+    """group_quantize_mxfp8_dbias rejects what it cannot do before any CUDA
+    call; its workspace is int64[G+1] block offsets padded to 256 bytes plus
+    fp32 [ceil(rows/32) + G, cols] block partials."""
+    lib = gl.load()
+    assert lib.gl_dbias_workspace_bytes(100, 64, 3) == 256 + (4 + 3) * 64 * 4
+    assert lib.gl_dbias_workspace_bytes(0, 64, 40) == 512 + 40 * 64 * 4
+    assert lib.gl_dbias_workspace_bytes(100, 0, 3) == 0
+    assert lib.gl_dbias_workspace_bytes(100, 64, 0) == 0
+    db = gl.GlGrouped(gl.GL_STACKED, 16, None)
+    ws = lib.gl_dbias_workspace_bytes(64, 128, 2)
+    f = lib.group_quantize_mxfp8_dbias
+    # row offsets, status and workspace are required
+    assert f(16, 64, 128, None, 2, 16, 16, 16, None, None, 0, db, 256, ws, None) == gl.GL_ERR_INVALID
+    assert f(16, 64, 128, 16, 2, None, 16, 16, None, None, 0, db, 256, ws, None) == gl.GL_ERR_INVALID
+    assert f(16, 64, 128, 16, 2, 16, 16, 16, None, None, 0, db, None, ws, None) == gl.GL_ERR_INVALID
+    # workspace too small / not 256-byte aligned
+    assert f(16, 64, 128, 16, 2, 16, 16, 16, None, None, 0, db, 256, ws - 1, None) == gl.GL_ERR_INVALID
+    assert f(16, 64, 128, 16, 2, 16, 16, 16, None, None, 0, db, 272, ws, None) == gl.GL_ERR_UNSUPPORTED
+    # dbias output missing; the cast's own checks still apply
+    assert f(16, 64, 128, 16, 2, 16, 16, 16, None, None, 0, gl.GlGrouped(gl.GL_STACKED, None, None), 256, ws,
+             None) == gl.GL_ERR_INVALID
+    assert f(16, 64, 48, 16, 2, 16, 16, 16, None, None, 0, db, 256, ws, None) == gl.GL_ERR_UNSUPPORTED
+
+
 def test_scale_bytes_helper():
     """Sizes of the scale arrays (host only): row-major [rows, cols/32] and
     [ceil(rows/32) + G, cols]; MMA layout in 512-byte atoms of 128 rows x 4
