@@ -291,6 +291,36 @@ gl_status group_quantize_mxfp8_dbias(const void* src, int64_t rows, int cols, co
 size_t gl_dbias_workspace_bytes(int64_t rows, int cols, int G);
 
 /*
+ * group_quantize_mxfp8_dbias_noalloc -- group_quantize_mxfp8_dbias for
+ * callers that cannot allocate device memory where they call it (their
+ * memory belongs to another runtime's pool and they are handed no allocator;
+ * a cudaMalloc there would also synchronise the device).  This entry point
+ * has no counterpart in the pages: it exists for those callers only.
+ *
+ * It takes no workspace: its scratch is one fixed 16 MiB array in the
+ * library's own device memory, which every GPU that loads the library holds
+ * until the process exits.  Every other argument, and the results, are those
+ * of group_quantize_mxfp8_dbias.
+ *   - gl_dbias_workspace_bytes(rows, cols, G) must be at most 16 MiB
+ *     (16777216): e.g. up to 9088 rows of 14336 columns in 8 groups, or
+ *     32000 rows of 4096 columns; larger calls return GL_ERR_UNSUPPORTED and
+ *     touch nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current) and may load the library's device code;
+ *     make that first call before any stream capture.  GL_ERR_CUDA if the
+ *     address cannot be obtained.
+ *   - Every call on a device uses the same array: calls whose work can
+ *     overlap on the GPU (other streams, or other threads' streams) race
+ *     and corrupt each other's results; order them on one stream or with
+ *     events.  No part of the array needs to start at zero.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+gl_status group_quantize_mxfp8_dbias_noalloc(const void* src, int64_t rows, int cols, const int64_t* row_offsets,
+                                             int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
+                                             uint8_t* codes_c, uint8_t* scales_c, int scale_layout,
+                                             gl_grouped dbias, void* stream);
+
+/*
  * MXFP8 grouped GEMMs -- the three products of gl_fwd / gl_dgrad / gl_wgrad
  * on MXFP8 operands (E4M3 codes, E8M0 scale per 32 contraction elements, as
  * written by group_quantize_mxfp8), computed as
