@@ -39,9 +39,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernels at the bench workload (profiles/step_bf16_g8_launch_list.md); an
 # entry must be removed when its kernel changes.
 MEASURED_TRAFFIC = {
-    "bf16_g8": {"fwd": 2858529280, "dgrad": 4030283264, "wgrad": 5714971904,
-                "quant_x": 217923072, "quant_w": 1878836224, "quant_dy": 910053376,
-                "fwd_mx": 1241643008, "dgrad_mx": 1571456000, "wgrad_mx": 3585101568},
+    "bf16_g8": {"fwd": 2548229120, "dgrad": 3429313792, "wgrad": 5650189824,
+                "quant_x": 218453760, "quant_w": 1878359296, "quant_dy": 910437120,
+                "fwd_mx": 1217792000, "dgrad_mx": 1443250944, "wgrad_mx": 3581297664},
 }
 
 
