@@ -21,7 +21,8 @@
 // relay (peer), warps 2-5 epilogue (TMEM -> registers; bias + bf16 rounding
 // and row-clipped stores for FWD/DGRAD; for WGRAD 32 x 32 fp32 chunks
 // transposed through shared memory and added into main_grad with coalesced
-// 16-byte vector reductions, or stored).  Two accumulators in TMEM let a tile's
+// 16-byte vector reductions, or stored; each tile's main_grad rows are first
+// pulled into L2 with bulk prefetches while its main loop runs).  Two accumulators in TMEM let a tile's
 // epilogue overlap the next tile's main loop.  Tiles are enumerated group by
 // group from the device offsets (tile prefix in shared memory): empty groups
 // cost nothing and the host never learns the split sizes.

@@ -15,7 +15,8 @@
 // MMAs overlap the stores.  wgrad: TN = 192 and two accumulators (384
 // columns); eight epilogue warps (half the columns each) transpose 32 x 32
 // fp32 chunks through shared memory and add them into main_grad with
-// coalesced 16-byte vector reductions.  The remaining TMEM columns hold the
+// coalesced 16-byte vector reductions (each tile's main_grad rows first
+// pulled into L2 with bulk prefetches).  The remaining TMEM columns hold the
 // scale-factor slots.
 //
 // Per stage (128 contraction elements = four MMAs of K=32) the producer
