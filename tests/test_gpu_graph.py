@@ -9,7 +9,6 @@ device buffer, and (the weight-cast ``noop`` use of ``grouped_linear.py``'s
 quantizers, PR #3224 "Improve device-init grouped linear module") skip a
 cast whose status word is set.
 """
-import numpy as np
 import pytest
 import torch
 
