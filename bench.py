@@ -527,6 +527,26 @@ def main():
         "note": "MXFP8 cast of dy (rowwise + columnwise) with its bias gradient in one pass; separate_ms = the "
                 "step's cast of dy + gl_dbias on the same splits; not part of the step"}
 
+    # The whole step captured once as a CUDA graph and replayed (every entry
+    # point is asynchronous, allocates nothing and never syncs the host), its
+    # device time beside the eager step's.
+    try:
+        g_stream = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(g_stream):
+            with torch.cuda.graph(graph, stream=g_stream):
+                step.run()
+        graph_ms = timed(graph.replay)
+        eager_ms = timed(step.run)  # the same 20-step burst, eager, right after
+        line["extras"]["graph_step"] = {"ms": graph_ms, "eager_ms": eager_ms,
+                                        "note": "one captured step replayed 20 times against 20 eager steps "
+                                                "right after (short bursts: clocks differ from the timed "
+                                                "region's); not the headline"}
+        del graph
+    except RuntimeError as exc:  # report, keep the line
+        line["extras"]["graph_step"] = {"unavailable": str(exc).splitlines()[0][:200]}
+
     # end to end on every rank (host buffers in, status out), slowest rank's time
     if world > 1:
         torch.distributed.barrier()

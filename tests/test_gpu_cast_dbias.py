@@ -137,3 +137,30 @@ def test_cast_dbias_full_size_bf16_g8_repeatable():
     _, db2 = gl.group_quantize_mxfp8_dbias(dy, off, st, mma_scales=True, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(db, db2)
+
+
+def test_many_groups_per_group_outputs():
+    """130 groups with per-group bias-gradient pointers: the reduction runs in
+    launches of 64 groups; the fused call and gl_dbias both match the oracle,
+    including the empty groups."""
+    rng = np.random.default_rng(130)
+    m = rng.integers(0, 40, size=130)
+    m[[3, 64, 65, 129]] = 0
+    G, M, N = len(m), int(m.sum()), 256
+    g = torch.Generator().manual_seed(130)
+    dy = torch.randn(M, N, generator=g).to(torch.bfloat16).cuda()
+    off, st = offsets_on_device(m, M)
+    fused = [torch.full((N,), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+    alone = [torch.full((N,), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+    gl.group_quantize_mxfp8_dbias(dy, off, st, mma_scales=True, dbias=fused)
+    gl.gl_dbias(dy, off, st, alone)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = orc.dbias(f64(dy), m)
+    for i in range(G):
+        for t in (fused[i], alone[i]):
+            got = f64(t)
+            if m[i] == 0:
+                assert np.all(got == 0.0), i
+            else:
+                assert orc.rel_frobenius(got, ref[i]) <= TOL_BF16, i
