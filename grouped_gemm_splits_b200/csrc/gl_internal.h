@@ -64,7 +64,7 @@ struct MxCall {
   int64_t M;
   int N, K;
   int accumulate;
-  int cta_pair;  // 1: 256x192 tiles on CTA pairs; 0: 128x192 tiles per CTA
+  int cta_pair;  // 1: CTA pairs (256x256 fprop/dgrad, 256x192 wgrad tiles); 0: single CTAs (128x256 / 128x192)
   cudaStream_t stream;
 };
 

@@ -10,7 +10,9 @@
  * ---------------------------------------
  *  - All tensors are row-major and contiguous; pointers named "device" point
  *    to memory of the current CUDA device; the caller owns every buffer.  The
- *    library never allocates device or pinned memory.
+ *    library never allocates device or pinned memory (the one scratch array
+ *    of group_quantize_mxfp8_dbias_noalloc is part of the library's device
+ *    image, not an allocation).
  *  - Shapes: x [M,K], W_i [N,K], b_i [N], y [y_rows,N], dy [M,N],
  *    dx [dx_rows,K], main_grad_i [N,K] fp32.  Group i owns rows
  *    [o[i], o[i+1]) of x, y, dy and dx, where o = offsets from gl_offsets.
@@ -86,7 +88,8 @@ const char* gl_status_string(gl_status s);
  * this process.  With GL_PAIRS_BF16 set the bf16 GEMMs compute 256 x 256
  * output tiles on pairs of CTAs (tcgen05 cta_group::2, one CTA per SM), else
  * 128 x 256 tiles on single CTAs.  With GL_PAIRS_MXFP8 set the MXFP8 GEMMs
- * compute 256 x 192 tiles on CTA pairs, else 128 x 192 tiles on single CTAs.
+ * compute 256 x 256 tiles (fprop, dgrad) and 256 x 192 tiles (wgrad) on CTA
+ * pairs, else 128 x 256 / 128 x 192 tiles on single CTAs.
  * Both flags are set by default.  Results agree within rounding.  Returns
  * GL_ERR_INVALID for unknown flag bits.
  */
