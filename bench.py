@@ -1,11 +1,19 @@
 """Benchmark of the grouped linear hot path on B200.
 
-One step = gl_offsets + gl_fwd + gl_dgrad + gl_wgrad (accumulate into fp32
-main_grad) over one batch of the ``bf16_g8`` workload (G=8 experts, K=4096,
-N=14336, 16384 rows split Multinomial(Dirichlet(1))), stacked [G,N,K] bf16
-weights resident in HBM.  ``value`` is whole-job TFLOP/s (the three GEMMs'
-2*sum(m)*N*K flops each, over all ranks, divided by the max-over-ranks device
-time of exactly ``--steps`` steps).
+One step = the whole path over one batch of the ``bf16_g8`` workload (G=8
+experts, K=4096, N=14336, 16384 rows split Multinomial(Dirichlet(1))), with
+stacked [G,N,K] bf16 weights and the fp32 main_grad resident in HBM:
+gl_offsets, bf16 gl_fwd / gl_dgrad / gl_wgrad (accumulate), then the MXFP8
+half on the ``mxfp8_g8`` splits (multiples of 128): group_quantize_mxfp8 of
+x, W and dy (rowwise + columnwise) and the three block-scaled GEMMs.
+``value`` is whole-job TFLOP/s: the six GEMMs' 2*sum(m)*N*K flops each, over
+all ranks, divided by the max-over-ranks device time of exactly ``--steps``
+steps.  ``--workload`` runs the same step at another workload's sizes and
+split sizes (its MXFP8 half on the same splits).
+
+Per-op times are medians over at least 50 steps (the timed ones, then untimed
+ones right after the timed region when ``--steps`` < 50), each op bracketed by
+CUDA events on the launching stream.
 
 Contract: ``python bench.py --gpus N --steps K --warmup W`` (torchrun for
 N > 1, one rank per GPU, every rank an independent replica: weak scaling);
@@ -15,6 +23,8 @@ numpy) on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import os
 import statistics
@@ -33,15 +43,40 @@ from grouped_gemm_splits_b200 import gl, synth  # noqa: E402
 METRIC = "grouped-GEMM TFLOPS fwd/dgrad/wgrad and % of B200 dense BF16/MXFP8 peak"
 WORKLOAD = "bf16_g8"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+OP_SAMPLES = 50  # per-op medians are taken over at least this many steps
 
-# DRAM bytes (read + write) per launch from one ncu capture of the current
-# kernels at the bench workload (profiles/step_bf16_g8_launch_list.md); an
-# entry must be removed when its kernel changes.
+# DRAM bytes (read + write) per launch of each kernel at a workload, from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the digest
+# of the CUDA sources the capture ran.  When the sources have changed since,
+# the figures describe other kernels: the line then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "bf16_g8": {"fwd": 2548229120, "dgrad": 3429313792, "wgrad": 5650189824,
-                "quant_x": 218453760, "quant_w": 1878359296, "quant_dy": 910437120,
-                "fwd_mx": 1217792000, "dgrad_mx": 1443250944, "wgrad_mx": 3581297664},
+    "csrc_digest": None,
 }
+
+
+def csrc_digest() -> str:
+    """Digest of the library's CUDA sources (names and contents)."""
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "grouped_gemm_splits_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(d, "*.cu")) + glob.glob(os.path.join(d, "*.cuh"))
+                    + glob.glob(os.path.join(d, "*.h"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, op: str):
+    """(bytes, source note) for a kernel, or (None, why not)."""
+    cap = MEASURED_TRAFFIC.get("csrc_digest")
+    if cap is None:
+        return None, "no ncu capture recorded for the current kernels"
+    if cap != csrc_digest():
+        return None, f"stale: the CUDA sources changed since the ncu capture ({cap})"
+    v = MEASURED_TRAFFIC.get(workload, {}).get(op)
+    if v is None:
+        return None, f"no ncu capture of this kernel at {workload}"
+    return v, f"ncu capture of sources {cap}"
 
 
 def peaks():
@@ -149,14 +184,17 @@ class MxStep:
             "dgrad_mx": code_b(M * N) + code_b(ne * N * K) + M * K * 2,
             "wgrad_mx": code_b(M * K) + code_b(M * N) + 2 * ne * N * K * 4,
         }
-        self.launches = 6
+        self.launches = 7  # offsets, three casts, three GEMMs
+
+    def run_offsets(self):
+        gl.gl_offsets(self.m_dev, self.wl.rows, self.wl.rows, self.offsets, self.status)
 
     def run(self, ev=None, i0=0):
+        """The casts and GEMMs (after ``run_offsets``); events ev[i0..i0+6]."""
         wl = self.wl
         G, N, K = wl.G, wl.N, wl.K
         if ev:
             ev[i0].record()
-        gl.gl_offsets(self.m_dev, wl.rows, wl.rows, self.offsets, self.status)
         gl.group_quantize_mxfp8(self.x, self.offsets, rowwise=True, colwise=True, status=self.status,
                                 out=self.qx, mma_scales=True)
         if ev:
@@ -211,12 +249,13 @@ class Step:
         self.names = ["offsets", "fwd", "dgrad", "wgrad"] + MxStep.NAMES
         self.flops = {"fwd": flops, "dgrad": flops, "wgrad": flops,
                       "fwd_mx": self.mx.flops, "dgrad_mx": self.mx.flops, "wgrad_mx": self.mx.flops}
-        self.bytes = {"offsets": G * 8 + (G + 1) * 8 + 4,
+        Gm = self.mx.wl.G
+        self.bytes = {"offsets": G * 8 + (G + 1) * 8 + 4 + Gm * 8 + (Gm + 1) * 8 + 4,
                       "fwd": xb + wb + dyb, "dgrad": dyb + wb + xb, "wgrad": xb + dyb + 2 * mgb}
         self.bytes.update(self.mx.bytes)
         self.dtype = {"fwd": "bf16", "dgrad": "bf16", "wgrad": "bf16",
                       "fwd_mx": "mxfp8", "dgrad_mx": "mxfp8", "wgrad_mx": "mxfp8"}
-        self.launches = 4 + self.mx.launches
+        self.launches = 4 + self.mx.launches  # offsets, fwd, dgrad, wgrad + the MXFP8 half
         self.total_flops = sum(self.flops.values())
 
     def run(self, ev=None):
@@ -224,6 +263,7 @@ class Step:
         if ev:
             ev[0].record()
         gl.gl_offsets(self.m_dev, self.wl.rows, self.wl.out_rows, self.offsets, self.status)
+        self.mx.run_offsets()  # the MXFP8 half's split sizes
         if ev:
             ev[1].record()
         gl.gl_fwd(self.x, self.w, self.bias, self.offsets, self.status, self.y)
@@ -413,7 +453,10 @@ def main():
     pk = peaks()
 
     nev = len(step.names) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    # per-op samples: the timed steps, plus untimed steps right after them
+    # until there are at least OP_SAMPLES (per-op medians)
+    n_samples = max(args.steps, OP_SAMPLES)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n_samples)]
     sampler = ClockSampler(local)
     sampler.start()  # sample clocks through warm-up and the timed region
     for _ in range(max(args.warmup, 3)):
@@ -433,10 +476,14 @@ def main():
     clocks = sampler.stop()
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
     ms_step = ms_total / args.steps
+    for i in range(args.steps, n_samples):  # outside the timed region
+        step.run(evs[i])
+    torch.cuda.synchronize()
     status = int(step.status.item()) | int(step.mx.status.item())
 
-    op_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
-             for j, n in enumerate(step.names)}
+    samples = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n_samples)]
+               for j, n in enumerate(step.names)}
+    op_ms = {n: statistics.median(v) for n, v in samples.items()}
     timed_s = ms_total / 1e3
     sustained = timed_s > 1.0
     peak_bf16 = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
@@ -448,31 +495,34 @@ def main():
         sec = op_ms[n] / 1e3
         by = step.bytes[n]
         fl = step.flops.get(n, 0.0)
-        e = {"ms": op_ms[n], "gbs": by / sec / 1e9}
-        tr = MEASURED_TRAFFIC.get(args.workload, {}).get(n)
+        e = {"ms": op_ms[n], "ms_mean": statistics.mean(samples[n]), "samples": n_samples,
+             "gbs": by / sec / 1e9, "algorithmic_bytes": by}
+        tr, tr_src = measured_traffic(args.workload, n)
+        e["dram_traffic_bytes"] = tr
         if tr:
-            e["dram_traffic_bytes"] = tr
             e["traffic_over_algorithmic"] = tr / by
         if fl:
             pkt = peak_of[step.dtype[n]]
-            t_roof = max(fl / (pkt * 1e12), by / (pk["hbm_gbs"] * 1e9))
+            t_flops, t_bytes = fl / (pkt * 1e12), by / (pk["hbm_gbs"] * 1e9)
             e.update({"tflops": fl / sec / 1e12, "dtype": step.dtype[n], "peak_tflops": pkt,
-                      "frac_of_roofline": t_roof / sec, "frac_of_tensor_peak": fl / sec / 1e12 / pkt})
+                      "bound": "tensor" if t_flops >= t_bytes else "hbm",
+                      "frac_of_roofline": max(t_flops, t_bytes) / sec, "frac_of_tensor_peak": fl / sec / 1e12 / pkt})
         else:
-            e.update({"frac_of_hbm": by / sec / 1e9 / pk["hbm_gbs"]})
+            e.update({"bound": "hbm", "frac_of_hbm": by / sec / 1e9 / pk["hbm_gbs"]})
         ops[n] = e
     dom = max(step.names, key=lambda n: op_ms[n])
-    if step.flops.get(dom):
-        roof = {"bound": "tensor", "kernel": f"{dom}", "achieved": ops[dom]["tflops"],
+    tr, tr_src = measured_traffic(args.workload, dom)
+    if ops[dom]["bound"] == "tensor":
+        roof = {"bound": "tensor", "kernel": dom, "achieved": ops[dom]["tflops"],
                 "peak": peak_of[step.dtype[dom]], "unit": "TFLOP/s",
                 "frac": ops[dom]["tflops"] / peak_of[step.dtype[dom]],
-                "peak_source": f"{pk['source']} bf16 ({peak_kind})" + (" x2 for fp8" if step.dtype[dom] == "mxfp8" else ""),
-                "traffic": MEASURED_TRAFFIC.get(args.workload, {}).get(dom)}
+                "peak_source": f"{pk['source']} bf16 ({peak_kind})" + (" x2 for fp8" if step.dtype[dom] == "mxfp8" else "")}
     else:
         roof = {"bound": "hbm", "kernel": dom, "achieved": ops[dom]["gbs"], "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": ops[dom]["gbs"] / pk["hbm_gbs"],
-                "peak_source": f"{pk['source']} copy bandwidth",
-                "traffic": MEASURED_TRAFFIC.get(args.workload, {}).get(dom)}
+                "peak_source": f"{pk['source']} copy bandwidth"}
+    roof.update({"traffic": tr, "traffic_source": tr_src, "algorithmic_bytes": step.bytes[dom],
+                 "ms": op_ms[dom], "samples": n_samples})
     value = job_tflops(step.total_flops, world, ms_step)
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -551,7 +601,7 @@ def main():
     if world > 1:
         torch.distributed.barrier()
     step_b = Step(args.workload, seed_offset=rank + 1000, device=dev)  # second buffer set
-    ms_e2e, h2d, d2h, st2 = e2e_measure((step, step_b), max(3, args.steps // 2), 2)
+    ms_e2e, h2d, d2h, st2 = e2e_measure((step, step_b), max(20, args.steps), 3)
     del step_b
     ms_e2e = max_over_ranks(ms_e2e, dev)
     line["e2e"] = {"value": job_tflops(step.total_flops, world, ms_e2e), "unit": "TFLOP/s",

@@ -1,16 +1,23 @@
 // gl_api.cu -- the C ABI (include/gl.h): argument checks, then launches.
 // Nothing here allocates device memory or synchronises the host.
-#include <atomic>
-
 #include "gl_internal.h"
 
 namespace {
 
-// bit 0: bf16 GEMMs on CTA pairs; bit 1: MXFP8 GEMMs on CTA pairs (both on
-// by default).
-std::atomic<int> g_cta_pair{GL_PAIRS_BF16 | GL_PAIRS_MXFP8};
-
 using gl::GemmCall;
+
+// Per-call GEMM options (NULL = defaults: CTA pairs, the kernels' own 2 s
+// wait bound).  False for values the header does not define.
+bool read_opts(const gl_gemm_opts* o, int* cta_pair, uint64_t* wait_ns) {
+  *cta_pair = 1;
+  *wait_ns = 0;  // 0: the kernel's default bound
+  if (o == nullptr) return true;
+  if (o->tiles != GL_TILES_PAIR && o->tiles != GL_TILES_SINGLE) return false;
+  if (o->wait_limit_us > GL_WAIT_LIMIT_MAX_US) return false;
+  *cta_pair = (o->tiles == GL_TILES_PAIR) ? 1 : 0;
+  *wait_ns = static_cast<uint64_t>(o->wait_limit_us) * 1000u;
+  return true;
+}
 
 cudaStream_t to_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -51,7 +58,7 @@ gl_status check_gemm_dims(int G, int64_t M, int N, int K) {
 
 extern "C" {
 
-int gl_version(void) { return 100; }
+int gl_version(void) { return 200; }
 
 const char* gl_status_string(gl_status s) {
   switch (s) {
@@ -63,12 +70,6 @@ const char* gl_status_string(gl_status s) {
   return "unknown status";
 }
 
-gl_status gl_set_cta_pair(int flags) {
-  if (flags & ~(GL_PAIRS_BF16 | GL_PAIRS_MXFP8)) return GL_ERR_INVALID;
-  g_cta_pair.store(flags);
-  return GL_OK;
-}
-
 gl_status gl_offsets(const int64_t* m_splits, int G, int64_t expect_rows, int64_t out_rows,
                      int64_t* offsets, int32_t* status, void* stream) {
   if (m_splits == nullptr || offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
@@ -78,9 +79,12 @@ gl_status gl_offsets(const int64_t* m_splits, int G, int64_t expect_rows, int64_
 
 gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int64_t* offsets,
                  int32_t* status, int G, int64_t M, int N, int K, void* y, int64_t y_rows,
-                 void* stream) {
+                 const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
+  int pair = 1;
+  uint64_t wait_ns = 0;
+  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
   if ((x == nullptr && M > 0) || (y == nullptr && M > 0) || offsets == nullptr || status == nullptr)
     return GL_ERR_INVALID;
   if (!grouped_ok(w, G) || (bias != nullptr && !grouped_ok(*bias, G))) return GL_ERR_INVALID;
@@ -101,15 +105,19 @@ gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int6
   c.M = M;
   c.N = N;
   c.K = K;
-  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_BF16) ? 1 : 0;
+  c.cta_pair = pair;
+  c.wait_ns = wait_ns;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
 
 gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t* status, int G,
-                   int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream) {
+                   int64_t M, int N, int K, void* dx, int64_t dx_rows, const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
+  int pair = 1;
+  uint64_t wait_ns = 0;
+  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
   if ((dy == nullptr && M > 0) || (dx == nullptr && M > 0) || offsets == nullptr || status == nullptr)
     return GL_ERR_INVALID;
   if (!grouped_ok(w, G)) return GL_ERR_INVALID;
@@ -128,15 +136,19 @@ gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t
   c.M = M;
   c.N = N;
   c.K = K;
-  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_BF16) ? 1 : 0;
+  c.cta_pair = pair;
+  c.wait_ns = wait_ns;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
 
 gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_t* status, int G,
-                   int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream) {
+                   int64_t M, int N, int K, gl_grouped main_grad, int accumulate, const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
+  int pair = 1;
+  uint64_t wait_ns = 0;
+  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
   if ((x == nullptr && M > 0) || (dy == nullptr && M > 0) || offsets == nullptr || status == nullptr)
     return GL_ERR_INVALID;
   if (!grouped_ok(main_grad, G)) return GL_ERR_INVALID;
@@ -161,7 +173,8 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
   c.N = N;
   c.K = K;
   c.accumulate = accumulate ? 1 : 0;
-  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_BF16) ? 1 : 0;
+  c.cta_pair = pair;
+  c.wait_ns = wait_ns;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -180,9 +193,12 @@ static gl_status check_mx_dims(int G, int64_t M, int N, int K) {
 gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_grouped w_codes,
                        gl_grouped w_scales, const gl_grouped* bias, const int64_t* offsets,
                        int32_t* status, int G, int64_t M, int N, int K, void* y, int64_t y_rows,
-                       void* stream) {
+                       const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_mx_dims(G, M, N, K);
   if (st != GL_OK) return st;
+  int pair = 1;
+  uint64_t wait_ns = 0;
+  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
   if (((x_codes == nullptr || x_scales == nullptr || y == nullptr) && M > 0) || offsets == nullptr ||
       status == nullptr)
     return GL_ERR_INVALID;
@@ -208,16 +224,20 @@ gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_group
   c.M = M;
   c.N = N;
   c.K = K;
-  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_MXFP8) ? 1 : 0;
+  c.cta_pair = pair;
+  c.wait_ns = wait_ns;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
 
 gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_grouped w_codes_c,
                          gl_grouped w_scales_c, const int64_t* offsets, int32_t* status, int G,
-                         int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream) {
+                         int64_t M, int N, int K, void* dx, int64_t dx_rows, const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_mx_dims(G, M, N, K);
   if (st != GL_OK) return st;
+  int pair = 1;
+  uint64_t wait_ns = 0;
+  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
   if (((dy_codes == nullptr || dy_scales == nullptr || dx == nullptr) && M > 0) || offsets == nullptr ||
       status == nullptr)
     return GL_ERR_INVALID;
@@ -241,16 +261,20 @@ gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_g
   c.M = M;
   c.N = N;
   c.K = K;
-  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_MXFP8) ? 1 : 0;
+  c.cta_pair = pair;
+  c.wait_ns = wait_ns;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
 
 gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, const uint8_t* dy_codes_c,
                          const uint8_t* dy_scales_c, const int64_t* offsets, int32_t* status, int G,
-                         int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream) {
+                         int64_t M, int N, int K, gl_grouped main_grad, int accumulate, const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_mx_dims(G, M, N, K);
   if (st != GL_OK) return st;
+  int pair = 1;
+  uint64_t wait_ns = 0;
+  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
   if (((x_codes_c == nullptr || x_scales_c == nullptr || dy_codes_c == nullptr || dy_scales_c == nullptr) &&
        M > 0) ||
       offsets == nullptr || status == nullptr)
@@ -278,7 +302,8 @@ gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, co
   c.N = N;
   c.K = K;
   c.accumulate = accumulate ? 1 : 0;
-  c.cta_pair = (g_cta_pair.load() & GL_PAIRS_MXFP8) ? 1 : 0;
+  c.cta_pair = pair;
+  c.wait_ns = wait_ns;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
@@ -317,6 +342,26 @@ gl_status check_quantize_args(const void* src, int64_t rows, int cols, const int
   return GL_OK;
 }
 
+}  // namespace
+
+namespace gl {
+
+gl_status check_quantize_dbias_args(const void* src, int64_t rows, int cols, const int64_t* row_offsets, int G,
+                                    const int32_t* status, const uint8_t* codes_r, const uint8_t* scales_r,
+                                    const uint8_t* codes_c, const uint8_t* scales_c, int scale_layout,
+                                    const gl_grouped& dbias) {
+  const gl_status st =
+      check_quantize_args(src, rows, cols, row_offsets, G, codes_r, scales_r, codes_c, scales_c, scale_layout);
+  if (st != GL_OK) return st;
+  if (row_offsets == nullptr || status == nullptr) return GL_ERR_INVALID;
+  if (!grouped_ok(dbias, G)) return GL_ERR_INVALID;
+  return GL_OK;
+}
+
+}  // namespace gl
+
+namespace {
+
 // Workspace of the fused cast + bias gradient: the groups' first blocks
 // (int64[G+1], padded to 256 bytes), then the per-block column sums.
 size_t dbias_ws_head(int G) { return ((static_cast<size_t>(G) + 1) * 8 + 255) / 256 * 256; }
@@ -346,11 +391,10 @@ gl_status group_quantize_mxfp8_dbias(const void* src, int64_t rows, int cols, co
                                      int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                                      uint8_t* codes_c, uint8_t* scales_c, int scale_layout, gl_grouped dbias,
                                      void* workspace, size_t workspace_bytes, void* stream) {
-  const gl_status st =
-      check_quantize_args(src, rows, cols, row_offsets, G, codes_r, scales_r, codes_c, scales_c, scale_layout);
+  const gl_status st = gl::check_quantize_dbias_args(src, rows, cols, row_offsets, G, status, codes_r, scales_r,
+                                                     codes_c, scales_c, scale_layout, dbias);
   if (st != GL_OK) return st;
-  if (row_offsets == nullptr || status == nullptr || workspace == nullptr) return GL_ERR_INVALID;
-  if (!grouped_ok(dbias, G)) return GL_ERR_INVALID;
+  if (workspace == nullptr) return GL_ERR_INVALID;
   if (workspace_bytes < gl_dbias_workspace_bytes(rows, cols, G)) return GL_ERR_INVALID;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GL_ERR_UNSUPPORTED;
   cudaStream_t s = to_stream(stream);

@@ -85,6 +85,7 @@ struct GemmParams {
   int N, K;
   int has_bias;
   int accumulate;
+  uint64_t wait_ns;  // bound on each pipeline wait
 };
 
 template <bool PG>
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
       for (int t = pair; t < total && !*abort_flag; t += npairs) {
         const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
         for (int kb = 0; kb < tl.num_kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { report_abort(abort_flag, p.status); break; }
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.wait_ns)) { report_abort(abort_flag, p.status); break; }
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
@@ -335,13 +336,16 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
         }
       }
       // Do not leave while a TMA load may still be writing shared memory: wait
-      // (bounded) for the last stages this thread filled.
+      // for the last stages this thread filled.  On a pair the leader's stage
+      // also waits for the peer's relay, which an aborted peer never sends, so
+      // one 2 s budget covers the whole drain.
       const int inflight = issued < C::kStages ? issued : C::kStages;
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
       int s = stage;
       uint32_t ph = phase;
       for (int i = 0; i < inflight; ++i) {
         if (--s < 0) { s = C::kStages - 1; ph ^= 1u; }
-        mbar_wait_bounded(&full[s], ph);
+        mbar_wait_until(&full[s], ph, deadline);
       }
     }
   } else if (warp == 1) {
@@ -355,7 +359,7 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
         const int buf = it & 1;
         const uint32_t tph = (it >> 1) & 1;
         // every lane waits; the warp acts on a unanimous result
-        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], tph ^ 1u, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], tph ^ 1u, abort_flag, p.wait_ns))) {
           report_abort(abort_flag, p.status);
           break;
         }
@@ -367,8 +371,8 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
           // relaying; acquire at cluster scope so those writes are visible.
           const bool peer_zeroed = CG == 2 && MODE == kWgrad && kb == tl.num_kb - 1 &&
                                    static_cast<int>(tl.r1 - tl.r0) - kb * BK < BK;
-          const bool landed = peer_zeroed ? mbar_wait_acq_cluster(&full[stage], phase, abort_flag)
-                                          : mbar_wait(&full[stage], phase, abort_flag);
+          const bool landed = peer_zeroed ? mbar_wait_acq_cluster(&full[stage], phase, abort_flag, p.wait_ns)
+                                          : mbar_wait(&full[stage], phase, abort_flag, p.wait_ns);
           if (!__all_sync(0xffffffffu, landed)) {
             report_abort(abort_flag, p.status);
             ok = false;
@@ -433,7 +437,7 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
         const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
         bool ok = true;
         for (int kb = 0; kb < tl.num_kb; ++kb) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, p.wait_ns))) {
             report_abort(abort_flag, p.status);
             ok = false;
             break;
@@ -485,7 +489,7 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
         // slower on small groups)
         prefetch_mg(tl);
       }
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag, p.wait_ns));
       if (!ok) report_abort(abort_flag, p.status);
       if (!ok) break;
       tc_fence_after();
@@ -695,6 +699,7 @@ gl_status launch_mode(const GemmCall& c) {
   prm.N = c.N;
   prm.K = c.K;
   prm.accumulate = c.accumulate;
+  prm.wait_ns = c.wait_ns ? c.wait_ns : kWaitLimitNs;
   prm.has_bias = (MODE == kFwd && c.bias != nullptr) ? 1 : 0;
   const uint64_t Mrows = c.M > 0 ? static_cast<uint64_t>(c.M) : 1;  // a map needs >= 1 row
   bool ok = true;

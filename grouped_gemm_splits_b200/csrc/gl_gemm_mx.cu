@@ -110,6 +110,7 @@ struct MxParams {
   int N, K;
   int has_bias;
   int accumulate;
+  uint64_t wait_ns;  // bound on each pipeline wait
 };
 
 template <bool PG>
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
         const Tile tl = decode<MODE, CG>(t, prefix, p);
         const int n0 = tl.nt * TN;  // first B operand row of the tile
         for (int kb = 0; kb < tl.num_kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { report_abort(abort_flag, p.status); break; }
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.wait_ns)) { report_abort(abort_flag, p.status); break; }
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           uint8_t* sf = sb + C::kBAlloc;
@@ -392,12 +393,17 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
       }
+      // Do not leave while a TMA load may still be writing shared memory: wait
+      // for the last stages this thread filled.  On a pair the leader's stage
+      // also waits for the peer's relay, which an aborted peer never sends, so
+      // one 2 s budget covers the whole drain.
       const int inflight = issued < C::kStages ? issued : C::kStages;
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
       int s = stage;
       uint32_t ph = phase;
       for (int i = 0; i < inflight; ++i) {
         if (--s < 0) { s = C::kStages - 1; ph ^= 1u; }
-        mbar_wait_bounded(&full[s], ph);
+        mbar_wait_until(&full[s], ph, deadline);
       }
     }
   } else if (warp == 1) {
@@ -411,7 +417,7 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
         const Tile tl = decode<MODE, CG>(t, prefix, p);
         const int buf = it % C::kAccBufs;
         const uint32_t tph = (it / C::kAccBufs) & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], tph ^ 1u, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], tph ^ 1u, abort_flag, p.wait_ns))) {
           report_abort(abort_flag, p.status);
           break;
         }
@@ -430,8 +436,8 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
           // the peer zeroed rows of its stage before relaying: acquire at
           // cluster scope so those writes are visible to the pair's MMAs
           const bool peer_zeroed = CG == 2 && MODE == kWgrad && valid < BK;
-          const bool landed = peer_zeroed ? mbar_wait_acq_cluster(&full[stage], phase, abort_flag)
-                                          : mbar_wait(&full[stage], phase, abort_flag);
+          const bool landed = peer_zeroed ? mbar_wait_acq_cluster(&full[stage], phase, abort_flag, p.wait_ns)
+                                          : mbar_wait(&full[stage], phase, abort_flag, p.wait_ns);
           if (!__all_sync(0xffffffffu, landed)) {
             report_abort(abort_flag, p.status);
             ok = false;
@@ -500,7 +506,7 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
         const Tile tl = decode<MODE, CG>(t, prefix, p);
         bool ok = true;
         for (int kb = 0; kb < tl.num_kb; ++kb) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, p.wait_ns))) {
             report_abort(abort_flag, p.status);
             ok = false;
             break;
@@ -552,7 +558,7 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
         // slower on small groups)
         prefetch_mg(tl);
       }
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag, p.wait_ns));
       if (!ok) report_abort(abort_flag, p.status);
       if (!ok) break;
       tc_fence_after();
@@ -772,6 +778,7 @@ gl_status mx_mode(const MxCall& c) {
   prm.N = c.N;
   prm.K = c.K;
   prm.accumulate = c.accumulate;
+  prm.wait_ns = c.wait_ns ? c.wait_ns : kWaitLimitNs;
   prm.has_bias = (MODE == kFwd && c.bias != nullptr) ? 1 : 0;
   prm.offsets_all = c.offsets;
   const uint64_t M = c.M > 0 ? static_cast<uint64_t>(c.M) : 1;

@@ -40,6 +40,7 @@ struct GemmCall {
   int N, K;
   int accumulate;
   int cta_pair;  // 1: 256x256 tiles on CTA pairs (cta_group::2); 0: 128x256 tiles per CTA
+  uint64_t wait_ns;  // bound on each pipeline wait inside the kernel
   cudaStream_t stream;
 };
 
@@ -65,6 +66,7 @@ struct MxCall {
   int N, K;
   int accumulate;
   int cta_pair;  // 1: CTA pairs (256x256 fprop/dgrad, 256x192 wgrad tiles); 0: single CTAs (128x256 / 128x192)
+  uint64_t wait_ns;  // bound on each pipeline wait inside the kernel
   cudaStream_t stream;
 };
 
@@ -83,6 +85,13 @@ gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t
                           int G, int32_t* status, uint8_t* codes_r, uint8_t* scales_r,
                           uint8_t* codes_c, uint8_t* scales_c, int scale_layout, float* part,
                           int64_t part_blocks, int64_t* part_prefix, cudaStream_t stream);
+
+// Argument checks of group_quantize_mxfp8_dbias other than its workspace
+// (GL_OK when the call is valid).
+gl_status check_quantize_dbias_args(const void* src, int64_t rows, int cols, const int64_t* row_offsets, int G,
+                                    const int32_t* status, const uint8_t* codes_r, const uint8_t* scales_r,
+                                    const uint8_t* codes_c, const uint8_t* scales_c, int scale_layout,
+                                    const gl_grouped& dbias);
 
 // Bias gradient from the cast's partials: dbias_g[n] = sum over the blocks
 // [part_prefix[g], part_prefix[g+1]) of part[b, n], in block order, rounded

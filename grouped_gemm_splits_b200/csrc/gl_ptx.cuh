@@ -55,9 +55,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false if the
-// wait exceeded kWaitLimitNs or *abort became non-zero (another role gave up).
+// wait exceeded limit_ns or *abort became non-zero (another role gave up).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const volatile int* abort) {
+                                          const volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
@@ -65,7 +66,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
 }
@@ -75,6 +76,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+// Wait until the phase completes or %globaltimer passes `deadline_ns` (one
+// time budget shared by a sequence of drain waits).
+__device__ __forceinline__ bool mbar_wait_until(uint64_t* bar, uint32_t parity, uint64_t deadline_ns) {
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() > deadline_ns) return false;
   }
   return true;
 }
@@ -286,13 +296,14 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_
 
 // Bounded wait with cluster-scope acquire (pairs with the release above).
 __device__ __forceinline__ bool mbar_wait_acq_cluster(uint64_t* bar, uint32_t parity,
-                                                      const volatile int* abort) {
+                                                      const volatile int* abort,
+                                                      uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait_acq_cluster(bar, parity)) {
     if ((++spins & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
   return true;

@@ -23,7 +23,7 @@ GL_DEV_NEG_SPLIT, GL_DEV_SUM_MISMATCH, GL_DEV_OUT_OVERFLOW, GL_DEV_TIMEOUT = 1, 
 GL_STACKED, GL_PER_GROUP = 0, 1
 GL_SCALES_ROWMAJOR, GL_SCALES_MMA = 0, 1
 
-EXPORTED = ("gl_version", "gl_status_string", "gl_set_cta_pair", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
+EXPORTED = ("gl_version", "gl_status_string", "gl_offsets", "gl_fwd", "gl_dgrad", "gl_wgrad",
             "gl_dbias", "group_quantize_mxfp8", "gl_mxfp8_scale_bytes", "gl_dbias_workspace_bytes",
             "group_quantize_mxfp8_dbias", "gl_fwd_mxfp8", "gl_dgrad_mxfp8", "gl_wgrad_mxfp8")
 
@@ -31,6 +31,13 @@ EXPORTED = ("gl_version", "gl_status_string", "gl_set_cta_pair", "gl_offsets", "
 class GlGrouped(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("base", ctypes.c_void_p),
                 ("ptrs", ctypes.POINTER(ctypes.c_void_p))]
+
+
+GL_TILES_PAIR, GL_TILES_SINGLE = 0, 1
+
+
+class GlGemmOpts(ctypes.Structure):
+    _fields_ = [("tiles", ctypes.c_int), ("wait_limit_us", ctypes.c_uint32)]
 
 
 class GlError(RuntimeError):
@@ -53,16 +60,15 @@ def load() -> ctypes.CDLL:
     L.gl_version.restype = i32
     L.gl_status_string.restype = ctypes.c_char_p
     L.gl_status_string.argtypes = [i32]
-    L.gl_set_cta_pair.restype = i32
-    L.gl_set_cta_pair.argtypes = [i32]
     L.gl_offsets.restype = i32
     L.gl_offsets.argtypes = [vp, i32, i64, i64, vp, vp, vp]
     L.gl_fwd.restype = i32
-    L.gl_fwd.argtypes = [vp, GlGrouped, ctypes.POINTER(GlGrouped), vp, vp, i32, i64, i32, i32, vp, i64, vp]
+    op = ctypes.POINTER(GlGemmOpts)
+    L.gl_fwd.argtypes = [vp, GlGrouped, ctypes.POINTER(GlGrouped), vp, vp, i32, i64, i32, i32, vp, i64, op, vp]
     L.gl_dgrad.restype = i32
-    L.gl_dgrad.argtypes = [vp, GlGrouped, vp, vp, i32, i64, i32, i32, vp, i64, vp]
+    L.gl_dgrad.argtypes = [vp, GlGrouped, vp, vp, i32, i64, i32, i32, vp, i64, op, vp]
     L.gl_wgrad.restype = i32
-    L.gl_wgrad.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, vp]
+    L.gl_wgrad.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, op, vp]
     L.gl_dbias.restype = i32
     L.gl_dbias.argtypes = [vp, vp, vp, i32, i64, i32, GlGrouped, vp]
     L.group_quantize_mxfp8.restype = i32
@@ -76,11 +82,11 @@ def load() -> ctypes.CDLL:
                                              ctypes.c_size_t, vp]
     L.gl_fwd_mxfp8.restype = i32
     L.gl_fwd_mxfp8.argtypes = [vp, vp, GlGrouped, GlGrouped, ctypes.POINTER(GlGrouped), vp, vp, i32, i64, i32,
-                               i32, vp, i64, vp]
+                               i32, vp, i64, op, vp]
     L.gl_dgrad_mxfp8.restype = i32
-    L.gl_dgrad_mxfp8.argtypes = [vp, vp, GlGrouped, GlGrouped, vp, vp, i32, i64, i32, i32, vp, i64, vp]
+    L.gl_dgrad_mxfp8.argtypes = [vp, vp, GlGrouped, GlGrouped, vp, vp, i32, i64, i32, i32, vp, i64, op, vp]
     L.gl_wgrad_mxfp8.restype = i32
-    L.gl_wgrad_mxfp8.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, vp]
+    L.gl_wgrad_mxfp8.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, GlGrouped, i32, op, vp]
     _lib = L
     return L
 
@@ -118,14 +124,11 @@ def _shape_nk(w: TensorOrList):
     return tuple((w if isinstance(w, torch.Tensor) else w[0]).shape[-2:])
 
 
-GL_PAIRS_BF16, GL_PAIRS_MXFP8 = 1, 2
-
-
-def gl_set_cta_pair(bf16: bool = True, mxfp8: bool = True) -> None:
-    """Tile shape of later GEMM launches: CTA pairs (256-row tiles) or single
-    CTAs (128-row tiles), separately for the bf16 and the MXFP8 GEMMs."""
-    _check(load().gl_set_cta_pair((GL_PAIRS_BF16 if bf16 else 0) | (GL_PAIRS_MXFP8 if mxfp8 else 0)),
-           "gl_set_cta_pair")
+def _opts(pair: bool, wait_limit_us: int):
+    """Per-call GEMM options (``gl_gemm_opts``); None for the defaults."""
+    if pair and not wait_limit_us:
+        return None
+    return ctypes.pointer(GlGemmOpts(GL_TILES_PAIR if pair else GL_TILES_SINGLE, wait_limit_us))
 
 
 def gl_offsets(m_splits: torch.Tensor, expect_rows: int, out_rows: Optional[int] = None,
@@ -144,7 +147,7 @@ def gl_offsets(m_splits: torch.Tensor, expect_rows: int, out_rows: Optional[int]
 
 
 def gl_fwd(x: torch.Tensor, w: TensorOrList, bias: Optional[TensorOrList], offsets: torch.Tensor,
-           status: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+           status: torch.Tensor, y: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0) -> torch.Tensor:
     """y rows of group g = x rows of group g @ W_g^T (+ b_g).  ``y`` may be a
     caller buffer with more rows than x; only the valid rows are written."""
     G = offsets.numel() - 1
@@ -160,13 +163,13 @@ def gl_fwd(x: torch.Tensor, w: TensorOrList, bias: Optional[TensorOrList], offse
         bg, keep_b = _grouped(bias, G)
         bptr = ctypes.pointer(bg)
     _check(load().gl_fwd(x.data_ptr(), wg, bptr, offsets.data_ptr(), status.data_ptr(), G, M, N, K,
-                         y.data_ptr(), y.shape[0], _stream()), "gl_fwd")
+                         y.data_ptr(), y.shape[0], _opts(pair, wait_limit_us), _stream()), "gl_fwd")
     del keep_w, keep_b
     return y
 
 
 def gl_dgrad(dy: torch.Tensor, w: TensorOrList, offsets: torch.Tensor, status: torch.Tensor,
-             dx: Optional[torch.Tensor] = None) -> torch.Tensor:
+             dx: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0) -> torch.Tensor:
     """dx rows of group g = dy rows of group g @ W_g."""
     G = offsets.numel() - 1
     M, N = dy.shape
@@ -176,20 +179,20 @@ def gl_dgrad(dy: torch.Tensor, w: TensorOrList, offsets: torch.Tensor, status: t
         dx = torch.empty(M, K, dtype=torch.bfloat16, device=dy.device)
     wg, keep_w = _grouped(w, G)
     _check(load().gl_dgrad(dy.data_ptr(), wg, offsets.data_ptr(), status.data_ptr(), G, M, N, K,
-                           dx.data_ptr(), dx.shape[0], _stream()), "gl_dgrad")
+                           dx.data_ptr(), dx.shape[0], _opts(pair, wait_limit_us), _stream()), "gl_dgrad")
     del keep_w
     return dx
 
 
 def gl_wgrad(x: torch.Tensor, dy: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
-             main_grad: TensorOrList, accumulate: bool = True) -> TensorOrList:
+             main_grad: TensorOrList, accumulate: bool = True, pair: bool = True, wait_limit_us: int = 0) -> TensorOrList:
     """main_grad[g] (+)= dy_g^T @ x_g (fp32)."""
     G = offsets.numel() - 1
     M, K = x.shape
     N = dy.shape[1]
     mg, keep = _grouped(main_grad, G)
     _check(load().gl_wgrad(x.data_ptr(), dy.data_ptr(), offsets.data_ptr(), status.data_ptr(), G,
-                           M, N, K, mg, 1 if accumulate else 0, _stream()), "gl_wgrad")
+                           M, N, K, mg, 1 if accumulate else 0, _opts(pair, wait_limit_us), _stream()), "gl_wgrad")
     del keep
     return main_grad
 
@@ -327,7 +330,7 @@ def _grouped_any(t: TensorOrList, G: int):
 
 def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorOrList, w_scales: TensorOrList,
                  bias: Optional[TensorOrList], offsets: torch.Tensor, status: torch.Tensor,
-                 y: Optional[torch.Tensor] = None) -> torch.Tensor:
+                 y: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0) -> torch.Tensor:
     """fprop on MXFP8 operands: x rowwise codes [M,K] + scale atoms; W rowwise
     codes [G,N,K] (or G x [N,K]) + scale atoms (all scales ``mma_scales``)."""
     G = offsets.numel() - 1
@@ -342,7 +345,7 @@ def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorO
         bg, k3 = _grouped(bias, G)
         bptr = ctypes.pointer(bg)
     _check(load().gl_fwd_mxfp8(x_codes.data_ptr(), x_scales.data_ptr(), wc, ws, bptr, offsets.data_ptr(),
-                               status.data_ptr(), G, M, N, K, y.data_ptr(), y.shape[0], _stream()),
+                               status.data_ptr(), G, M, N, K, y.data_ptr(), y.shape[0], _opts(pair, wait_limit_us), _stream()),
            "gl_fwd_mxfp8")
     del k1, k2, k3
     return y
@@ -350,7 +353,7 @@ def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorO
 
 def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: TensorOrList,
                    w_scales_c: TensorOrList, offsets: torch.Tensor, status: torch.Tensor,
-                   dx: Optional[torch.Tensor] = None) -> torch.Tensor:
+                   dx: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0) -> torch.Tensor:
     """dgrad on MXFP8 operands: dy rowwise codes [M,N] + scale atoms; W
     columnwise codes [G,N,K] + columnwise scale atoms."""
     G = offsets.numel() - 1
@@ -361,7 +364,7 @@ def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: T
     wc, k1 = _grouped_any(w_codes_c, G)
     ws, k2 = _grouped_any(w_scales_c, G)
     _check(load().gl_dgrad_mxfp8(dy_codes.data_ptr(), dy_scales.data_ptr(), wc, ws, offsets.data_ptr(),
-                                 status.data_ptr(), G, M, N, K, dx.data_ptr(), dx.shape[0], _stream()),
+                                 status.data_ptr(), G, M, N, K, dx.data_ptr(), dx.shape[0], _opts(pair, wait_limit_us), _stream()),
            "gl_dgrad_mxfp8")
     del k1, k2
     return dx
@@ -369,7 +372,7 @@ def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: T
 
 def gl_wgrad_mxfp8(x_codes_c: torch.Tensor, x_scales_c: torch.Tensor, dy_codes_c: torch.Tensor,
                    dy_scales_c: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
-                   main_grad: TensorOrList, accumulate: bool = True) -> TensorOrList:
+                   main_grad: TensorOrList, accumulate: bool = True, pair: bool = True, wait_limit_us: int = 0) -> TensorOrList:
     """wgrad on MXFP8 operands: x and dy columnwise codes + columnwise scale atoms."""
     G = offsets.numel() - 1
     M, K = x_codes_c.shape
@@ -377,6 +380,6 @@ def gl_wgrad_mxfp8(x_codes_c: torch.Tensor, x_scales_c: torch.Tensor, dy_codes_c
     mg, keep = _grouped(main_grad, G)
     _check(load().gl_wgrad_mxfp8(x_codes_c.data_ptr(), x_scales_c.data_ptr(), dy_codes_c.data_ptr(),
                                  dy_scales_c.data_ptr(), offsets.data_ptr(), status.data_ptr(), G, M, N, K, mg,
-                                 1 if accumulate else 0, _stream()), "gl_wgrad_mxfp8")
+                                 1 if accumulate else 0, _opts(pair, wait_limit_us), _stream()), "gl_wgrad_mxfp8")
     del keep
     return main_grad

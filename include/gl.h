@@ -84,18 +84,33 @@ int gl_version(void);
 const char* gl_status_string(gl_status s);
 
 /*
- * gl_set_cta_pair -- tile shape of the grouped GEMMs launched afterwards by
- * this process.  With GL_PAIRS_BF16 set the bf16 GEMMs compute 256 x 256
- * output tiles on pairs of CTAs (tcgen05 cta_group::2, one CTA per SM), else
- * 128 x 256 tiles on single CTAs.  With GL_PAIRS_MXFP8 set the MXFP8 GEMMs
- * compute 256 x 256 tiles (fprop, dgrad) and 256 x 192 tiles (wgrad) on CTA
- * pairs, else 128 x 256 / 128 x 192 tiles on single CTAs.
- * Both flags are set by default.  Results agree within rounding.  Returns
- * GL_ERR_INVALID for unknown flag bits.
+ * gl_gemm_opts -- per-call options of the six grouped GEMMs (gl_fwd,
+ * gl_dgrad, gl_wgrad and their MXFP8 forms); pass NULL for the defaults.
+ * They belong to the one call: the library keeps no mode between calls, so
+ * callers on different threads never change each other's kernels.
+ *
+ *   tiles          GL_TILES_PAIR (0, the default): 256-row output tiles on
+ *                  pairs of CTAs (tcgen05 cta_group::2, one CTA per SM) --
+ *                  bf16 256 x 256; MXFP8 256 x 256 (fprop, dgrad) and
+ *                  256 x 192 (wgrad).  GL_TILES_SINGLE: 128-row tiles on
+ *                  single CTAs (bf16 128 x 256; MXFP8 128 x 256 and
+ *                  128 x 192).  Results agree within rounding.
+ *   wait_limit_us  bound, in microseconds, on each wait of the kernel's
+ *                  load -> MMA -> epilogue pipeline; 0 = the default (2 s),
+ *                  at most GL_WAIT_LIMIT_MAX_US.  A wait that runs out ORs
+ *                  GL_DEV_TIMEOUT into the status word and the kernel stops
+ *                  early with its outputs incomplete.  It exists to exercise
+ *                  that failure path; the waits that drain a CTA's in-flight
+ *                  copies and MMAs before it exits keep their 2 s bound.
+ * Values the header does not define give GL_ERR_INVALID.
  */
-#define GL_PAIRS_BF16 1
-#define GL_PAIRS_MXFP8 2
-gl_status gl_set_cta_pair(int flags);
+#define GL_TILES_PAIR 0
+#define GL_TILES_SINGLE 1
+#define GL_WAIT_LIMIT_MAX_US 2000000u
+typedef struct gl_gemm_opts {
+  int tiles;
+  uint32_t wait_limit_us;
+} gl_gemm_opts;
 
 /*
  * gl_offsets -- group row offsets from the split sizes, on the device.
@@ -132,13 +147,14 @@ gl_status gl_offsets(const int64_t* m_splits, int G, int64_t expect_rows, int64_
  *   offsets  device int64[G+1] from gl_offsets
  *   status   device int32 status word from gl_offsets (read; may get TIMEOUT)
  *   y        device bf16 [y_rows, N], y_rows >= M
+ *   opts     NULL (defaults) or per-call options, see gl_gemm_opts
  * Limits: K % 8 == 0, N % 8 == 0 (16-byte row pitch), G <= GL_MAX_GROUPS.
  * The bias is added to the fp32 accumulator, then one round-to-nearest-even
  * conversion gives the bf16 output.
  */
 gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int64_t* offsets,
                  int32_t* status, int G, int64_t M, int N, int K, void* y, int64_t y_rows,
-                 void* stream);
+                 const gl_gemm_opts* opts, void* stream);
 
 /*
  * gl_dgrad -- grouped data gradient, dx_i = dy_i W_i.
@@ -153,7 +169,7 @@ gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int6
  * Limits: K % 8 == 0, N % 8 == 0.
  */
 gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t* status, int G,
-                   int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream);
+                   int64_t M, int N, int K, void* dx, int64_t dx_rows, const gl_gemm_opts* opts, void* stream);
 
 /*
  * gl_wgrad -- grouped weight gradient into fp32 main_grad.
@@ -170,7 +186,7 @@ gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t
  * Limits: K % 8 == 0, N % 8 == 0.
  */
 gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_t* status, int G,
-                   int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream);
+                   int64_t M, int N, int K, gl_grouped main_grad, int accumulate, const gl_gemm_opts* opts, void* stream);
 
 /*
  * gl_dbias -- bias gradient: db_i[n] = sum of dy[r, n] over the rows r of
@@ -304,14 +320,20 @@ size_t gl_dbias_workspace_bytes(int64_t rows, int cols, int G);
  * library's own device memory, which every GPU that loads the library holds
  * until the process exits.  Every other argument, and the results, are those
  * of group_quantize_mxfp8_dbias.
- *   - gl_dbias_workspace_bytes(rows, cols, G) must be at most 16 MiB
- *     (16777216): e.g. up to 9088 rows of 14336 columns in 8 groups, or
- *     32000 rows of 4096 columns; larger calls return GL_ERR_UNSUPPORTED and
- *     touch nothing.
+ *   - gl_dbias_workspace_bytes(rows, cols, G), which is
+ *     256 * ceil(8 (G + 1) / 256) + 4 * cols * (ceil(rows / 32) + G),
+ *     must be at most 16 MiB (16777216): e.g. up to 9088 rows of 14336
+ *     columns in 8 groups, or 32000 rows of 4096 columns in at most 23
+ *     groups.  Larger calls return GL_ERR_UNSUPPORTED and touch nothing;
+ *     argument errors are reported first, as group_quantize_mxfp8_dbias
+ *     reports them.
  *   - The first call on each device looks up the array's device address
  *     (with that device current) and may load the library's device code;
- *     make that first call before any stream capture.  GL_ERR_CUDA if the
- *     address cannot be obtained.
+ *     make that first call before any stream capture.  The address is kept
+ *     with the identity of its CUDA context, so after a device reset the next
+ *     call looks it up again.  GL_ERR_CUDA if the address cannot be obtained
+ *     (the runtime's last-error state is cleared, so later calls are not
+ *     affected).
  *   - Every call on a device uses the same array: calls whose work can
  *     overlap on the GPU (other streams, or other threads' streams) race
  *     and corrupt each other's results; order them on one stream or with
@@ -350,15 +372,15 @@ gl_status group_quantize_mxfp8_dbias_noalloc(const void* src, int64_t rows, int 
 gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_grouped w_codes,
                        gl_grouped w_scales, const gl_grouped* bias, const int64_t* offsets,
                        int32_t* status, int G, int64_t M, int N, int K, void* y, int64_t y_rows,
-                       void* stream);
+                       const gl_gemm_opts* opts, void* stream);
 
 gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_grouped w_codes_c,
                          gl_grouped w_scales_c, const int64_t* offsets, int32_t* status, int G,
-                         int64_t M, int N, int K, void* dx, int64_t dx_rows, void* stream);
+                         int64_t M, int N, int K, void* dx, int64_t dx_rows, const gl_gemm_opts* opts, void* stream);
 
 gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, const uint8_t* dy_codes_c,
                          const uint8_t* dy_scales_c, const int64_t* offsets, int32_t* status, int G,
-                         int64_t M, int N, int K, gl_grouped main_grad, int accumulate, void* stream);
+                         int64_t M, int N, int K, gl_grouped main_grad, int accumulate, const gl_gemm_opts* opts, void* stream);
 
 #ifdef __cplusplus
 }

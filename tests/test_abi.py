@@ -38,22 +38,22 @@ def test_host_side_validation_without_gpu():
     lib = gl.load()
     w = gl.GlGrouped(gl.GL_STACKED, 16, None)
     # G <= 0, N/K <= 0: ValueError analogues of GroupedLinear's constructor checks
-    assert lib.gl_fwd(16, w, None, 16, 16, 0, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
-    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 0, 8, 16, 8, None) == gl.GL_ERR_INVALID
+    assert lib.gl_fwd(16, w, None, 16, 16, 0, 8, 8, 8, 16, 8, None, None) == gl.GL_ERR_INVALID
+    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 0, 8, 16, 8, None, None) == gl.GL_ERR_INVALID
     # N % 8 != 0: unsupported row pitch
-    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 12, 8, 16, 8, None) == gl.GL_ERR_UNSUPPORTED
+    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 12, 8, 16, 8, None, None) == gl.GL_ERR_UNSUPPORTED
     # caller buffer with fewer rows than the input
-    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 8, 8, 16, 7, None) == gl.GL_ERR_INVALID
+    assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 8, 8, 16, 7, None, None) == gl.GL_ERR_INVALID
     # null pointers
-    assert lib.gl_fwd(None, w, None, 16, 16, 2, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
-    assert lib.gl_dgrad(16, w, 16, None, 2, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
-    assert lib.gl_wgrad(16, 16, 16, 16, 2, 8, 8, 8, gl.GlGrouped(gl.GL_STACKED, None, None), 1, None) == gl.GL_ERR_INVALID
+    assert lib.gl_fwd(None, w, None, 16, 16, 2, 8, 8, 8, 16, 8, None, None) == gl.GL_ERR_INVALID
+    assert lib.gl_dgrad(16, w, 16, None, 2, 8, 8, 8, 16, 8, None, None) == gl.GL_ERR_INVALID
+    assert lib.gl_wgrad(16, 16, 16, 16, 2, 8, 8, 8, gl.GlGrouped(gl.GL_STACKED, None, None), 1, None, None) == gl.GL_ERR_INVALID
     assert lib.gl_offsets(None, 4, 8, 8, 16, 16, None) == gl.GL_ERR_INVALID
     assert lib.gl_offsets(16, 0, 8, 8, 16, 16, None) == gl.GL_ERR_INVALID
     # per-group mode with a null member pointer
     arr = (ctypes.c_void_p * 2)(16, None)
     pg = gl.GlGrouped(gl.GL_PER_GROUP, None, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
-    assert lib.gl_fwd(16, pg, None, 16, 16, 2, 8, 8, 8, 16, 8, None) == gl.GL_ERR_INVALID
+    assert lib.gl_fwd(16, pg, None, 16, 16, 2, 8, 8, 8, 16, 8, None, None) == gl.GL_ERR_INVALID
     # quantize: cols not a multiple of 32; no output requested
     assert lib.group_quantize_mxfp8(16, 8, 48, None, 1, None, 16, 16, None, None, 0, None) == gl.GL_ERR_UNSUPPORTED
     assert lib.group_quantize_mxfp8(16, 8, 64, None, 1, None, None, None, None, None, 0, None) == gl.GL_ERR_INVALID
@@ -66,6 +66,27 @@ def test_host_side_validation_without_gpu():
     # MMA-layout scales need cols % 128 == 0; unknown layout codes are rejected
     assert lib.group_quantize_mxfp8(16, 8, 96, None, 1, None, 16, 16, None, None, 1, None) == gl.GL_ERR_UNSUPPORTED
     assert lib.group_quantize_mxfp8(16, 8, 128, None, 1, None, 16, 16, None, None, 7, None) == gl.GL_ERR_INVALID
+
+
+def test_gemm_options_are_checked():
+    """Per-call GEMM options: tile choices and wait bounds the header does not
+    define are refused before any launch; the defaults (NULL) are accepted."""
+    lib = gl.load()
+    w = gl.GlGrouped(gl.GL_STACKED, 16, None)
+    bad_tiles = ctypes.pointer(gl.GlGemmOpts(7, 0))
+    too_long = ctypes.pointer(gl.GlGemmOpts(gl.GL_TILES_PAIR, 2000001))
+    for o in (bad_tiles, too_long):
+        assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 8, 8, 16, 8, o, None) == gl.GL_ERR_INVALID
+        assert lib.gl_dgrad(16, w, 16, 16, 2, 8, 8, 8, 16, 8, o, None) == gl.GL_ERR_INVALID
+        assert lib.gl_wgrad(16, 16, 16, 16, 2, 8, 8, 8, w, 1, o, None) == gl.GL_ERR_INVALID
+        assert lib.gl_fwd_mxfp8(16, 16, w, w, None, 16, 16, 2, 8, 128, 128, 16, 8, o, None) == gl.GL_ERR_INVALID
+        assert lib.gl_dgrad_mxfp8(16, 16, w, w, 16, 16, 2, 8, 128, 128, 16, 8, o, None) == gl.GL_ERR_INVALID
+        assert lib.gl_wgrad_mxfp8(16, 16, 16, 16, 16, 16, 2, 8, 128, 128, w, 1, o, None) == gl.GL_ERR_INVALID
+    # no rows: valid options (and NULL) return before any launch
+    ok = ctypes.pointer(gl.GlGemmOpts(gl.GL_TILES_SINGLE, 1))
+    for o in (None, ok):
+        assert lib.gl_fwd(16, w, None, 16, 16, 2, 0, 8, 8, 16, 0, o, None) == gl.GL_OK
+        assert lib.gl_dgrad(16, w, 16, 16, 2, 0, 8, 8, 16, 0, o, None) == gl.GL_OK
 
 
 def test_fused_cast_dbias_validation_and_workspace_size():

@@ -19,13 +19,11 @@ from tests.gpu_util import (TOL_BF16, assert_groups_close, f64, offsets_on_devic
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["pair", "single"])
-def tile_mode(request):
-    """Run a test with 256x256 tiles on CTA pairs and with 128x256 tiles on
-    single CTAs; the default (pairs) is restored afterwards."""
-    gl.gl_set_cta_pair(bf16=request.param == "pair")
-    yield request.param
-    gl.gl_set_cta_pair()  # defaults
+@pytest.fixture(params=[True, False], ids=["pair", "single"])
+def pair(request):
+    """256x256 tiles on CTA pairs, or 128x256 tiles on single CTAs (a per-call
+    option of every GEMM)."""
+    return request.param
 
 # (G, N, K, m_splits): several tiles, ragged tails in every dimension,
 # empty groups, groups shorter than one MMA step.
@@ -46,7 +44,7 @@ def _inputs(G, N, K, m, seed, bias=True, device="cuda"):
 
 @pytest.mark.parametrize("G,N,K,m", SMALL)
 @pytest.mark.parametrize("per_group", [False, True])
-def test_fwd_dgrad_wgrad_small(G, N, K, m, per_group, tile_mode):
+def test_fwd_dgrad_wgrad_small(G, N, K, m, per_group, pair):
     M = int(sum(m))
     d = _inputs(G, N, K, m, seed=G * 7 + N)
     off, st = offsets_on_device(m, M, M + 64)
@@ -55,14 +53,14 @@ def test_fwd_dgrad_wgrad_small(G, N, K, m, per_group, tile_mode):
     x64, w64, b64, dy64 = f64(d["x"]), f64(d["w"]), f64(d["bias"]), f64(d["dy"])
 
     y = sentinel_like(M + 64, N)
-    gl.gl_fwd(d["x"], w, b, off, st, y)
+    gl.gl_fwd(d["x"], w, b, off, st, y, pair=pair)
     dx = sentinel_like(M + 64, K)
-    gl.gl_dgrad(d["dy"], w, off, st, dx)
+    gl.gl_dgrad(d["dy"], w, off, st, dx, pair=pair)
     mg_acc = d["main_grad"].clone()
     mg_acc_arg = [mg_acc[i] for i in range(G)] if per_group else mg_acc
-    gl.gl_wgrad(d["x"], d["dy"], off, st, mg_acc_arg, accumulate=True)
+    gl.gl_wgrad(d["x"], d["dy"], off, st, mg_acc_arg, accumulate=True, pair=pair)
     mg_over = torch.full_like(d["main_grad"], float("nan"))
-    gl.gl_wgrad(d["x"], d["dy"], off, st, mg_over, accumulate=False)
+    gl.gl_wgrad(d["x"], d["dy"], off, st, mg_over, accumulate=False, pair=pair)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
 
@@ -83,17 +81,17 @@ def test_fwd_dgrad_wgrad_small(G, N, K, m, per_group, tile_mode):
             assert orc.rel_frobenius(got_over[g], ref_over[g]) <= TOL_BF16, g
 
 
-def test_integer_mode_bit_exact(tile_mode):
+def test_integer_mode_bit_exact(pair):
     """{-1,0,1} operands and integer biases: every sum is exact, so the GPU
     must reproduce the oracle bit for bit (tiny workload shapes)."""
     G, N, K, m = 4, 256, 128, [0, 96, 160, 256]
     M = sum(m)
     d = {k: v.cuda() for k, v in synth.integer_operands(G, M, N, K, seed=11).items()}
     off, st = offsets_on_device(m, M)
-    y = gl.gl_fwd(d["x"], d["w"], d["bias"], off, st)
-    dx = gl.gl_dgrad(d["dy"], d["w"], off, st)
+    y = gl.gl_fwd(d["x"], d["w"], d["bias"], off, st, pair=pair)
+    dx = gl.gl_dgrad(d["dy"], d["w"], off, st, pair=pair)
     mg = d["main_grad"].clone()
-    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True)
+    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True, pair=pair)
     torch.cuda.synchronize()
     x64, w64, b64, dy64 = f64(d["x"]), f64(d["w"]), f64(d["bias"]), f64(d["dy"])
     ref_y = orc.fwd(x64, w64, b64, m)
@@ -129,7 +127,7 @@ def test_caller_buffer_matches_internal_allocation():
     assert untouched(y_buf[M:])
 
 
-def test_many_groups_per_group_chunking(tile_mode):
+def test_many_groups_per_group_chunking(pair):
     """More groups than one launch carries in per-group mode (64)."""
     rng = np.random.default_rng(9)
     G, N, K = 150, 136, 64
@@ -138,9 +136,9 @@ def test_many_groups_per_group_chunking(tile_mode):
     d = _inputs(G, N, K, m, seed=9)
     off, st = offsets_on_device(m, M)
     wl = [d["w"][i].clone() for i in range(G)]
-    y = gl.gl_fwd(d["x"], wl, [d["bias"][i] for i in range(G)], off, st)
+    y = gl.gl_fwd(d["x"], wl, [d["bias"][i] for i in range(G)], off, st, pair=pair)
     mg = [d["main_grad"][i].clone() for i in range(G)]
-    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True)
+    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True, pair=pair)
     torch.cuda.synchronize()
     x64, w64, dy64 = f64(d["x"]), f64(d["w"]), f64(d["dy"])
     assert_groups_close(f64(y), orc.fwd(x64, w64, f64(d["bias"]), m), m)
@@ -152,19 +150,19 @@ def test_many_groups_per_group_chunking(tile_mode):
             assert orc.rel_frobenius(got[g] - mg0[g], ref[g] - mg0[g]) <= TOL_BF16
 
 
-def test_all_groups_empty(tile_mode):
+def test_all_groups_empty(pair):
     G, N, K, m = 3, 256, 128, [0, 0, 0]
     d = synth.operands(G, 8, N, K, 1)
     x = d["x"].cuda()[:0]      # zero rows, but a valid base pointer
     dy = d["dy"].cuda()[:0]
     off, st = offsets_on_device(m, 0, 16)
     y = sentinel_like(16, N)
-    gl.gl_fwd(x, d["w"].cuda(), None, off, st, y)
+    gl.gl_fwd(x, d["w"].cuda(), None, off, st, y, pair=pair)
     mg = d["main_grad"].cuda()
     mg0 = mg.clone()
-    gl.gl_wgrad(x, dy, off, st, mg, accumulate=True)
+    gl.gl_wgrad(x, dy, off, st, mg, accumulate=True, pair=pair)
     mgo = torch.full_like(mg, 3.0)
-    gl.gl_wgrad(x, dy, off, st, mgo, accumulate=False)
+    gl.gl_wgrad(x, dy, off, st, mgo, accumulate=False, pair=pair)
     torch.cuda.synchronize()
     assert untouched(y)
     assert torch.equal(mg, mg0)
@@ -189,72 +187,117 @@ def test_bad_splits_write_nothing():
 
 
 # ----------------------------------------------------------------------------
-# Full-size workloads, checked on sampled outputs one entry at a time
+# Full-size workloads, checked group by group on sampled outputs
 # ----------------------------------------------------------------------------
 
 FULL = ["bf16_g8", "fine_g64", "stacked_g128_uniform", "stacked_g128_ragged"]
+ROWS_PER_GROUP = 8   # random rows per group, besides the group's first and last row
+COLS = 64            # output columns sampled per group (fwd: of N, dgrad: of K)
+WG = 8               # wgrad: WG x WG sampled (n, k) entries per group
 
 
-def _sampled_parity(name):
+def _idx(v):
+    return torch.as_tensor(np.asarray(v, dtype=np.int64), device="cuda")
+
+
+def _sampled_parity(name, pair):
+    """Run fwd, dgrad and wgrad (accumulate) at full size, then check every
+    non-empty group on its own against the oracle's single-entry products:
+    its first, last and ROWS_PER_GROUP random rows x COLS random columns of y
+    and dx, and WG x WG entries of main_grad, each within 5e-3 relative
+    Frobenius error; empty groups keep main_grad bit-identical."""
     wl = synth.WORKLOADS[name]
     m = synth.m_splits_for(name)
     G, N, K, M = wl.G, wl.N, wl.K, wl.rows
     d = synth.operands(G, M, N, K, wl.seed, device="cuda", bias=wl.bias)
     off, st = offsets_on_device(m, M, wl.out_rows)
     y = sentinel_like(wl.out_rows, N)
-    gl.gl_fwd(d["x"], d["w"], d.get("bias"), off, st, y)
+    gl.gl_fwd(d["x"], d["w"], d.get("bias"), off, st, y, pair=pair)
     dx = sentinel_like(wl.out_rows, K)
-    gl.gl_dgrad(d["dy"], d["w"], off, st, dx)
+    gl.gl_dgrad(d["dy"], d["w"], off, st, dx, pair=pair)
     mg = d["main_grad"].clone()
-    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True)
+    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True, pair=pair)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert untouched(y[M:]) and untouched(dx[M:])
 
     rng = np.random.default_rng(wl.seed)
     o = orc.offsets(m)
-    rows = sample_rows(m, 3, rng)
-    grp = np.searchsorted(o, rows, side="right") - 1
-    ncols = 24
-    # fwd / dgrad: per sampled row, a random set of output columns
-    got_f, ref_f, got_d, ref_d = [], [], [], []
-    x_rows = f64(d["x"][torch.tensor(rows, device="cuda")])
-    dy_rows = f64(d["dy"][torch.tensor(rows, device="cuda")])
-    for j, r in enumerate(rows):
-        g = int(grp[j])
-        ns = rng.integers(0, N, size=ncols)
-        ks = rng.integers(0, K, size=ncols)
-        wr = f64(d["w"][g, torch.tensor(ns, device="cuda")])            # [ncols, K]
-        wc = f64(d["w"][g][:, torch.tensor(ks, device="cuda")]).T       # [ncols, N]
-        bias = f64(d["bias"][g]) if wl.bias else None
-        for i, n in enumerate(ns):
-            ref_f.append(orc.fwd_entry(x_rows[j], wr[i], None if bias is None else bias[n]))
-        got_f += list(f64(y[int(r), torch.tensor(ns, device="cuda")]))
-        for i, k in enumerate(ks):
-            ref_d.append(orc.dgrad_entry(dy_rows[j], wc[i]))
-        got_d += list(f64(dx[int(r), torch.tensor(ks, device="cuda")]))
-    assert orc.rel_frobenius(np.array(got_f), np.array(ref_f)) <= TOL_BF16
-    assert orc.rel_frobenius(np.array(got_d), np.array(ref_d)) <= TOL_BF16
-    # wgrad: sampled (g, n, k) entries of main_grad
-    got_w, ref_w = [], []
+    checked = 0
     for g in range(G):
         a, b = int(o[g]), int(o[g + 1])
         if a == b:
+            assert torch.equal(mg[g], d["main_grad"][g]), ("accumulate touched an empty group", g)
             continue
-        ns = rng.integers(0, N, size=4)
-        ks = rng.integers(0, K, size=4)
-        dyc = f64(d["dy"][a:b][:, torch.tensor(ns, device="cuda")])
-        xc = f64(d["x"][a:b][:, torch.tensor(ks, device="cuda")])
-        old = f64(d["main_grad"][g][torch.tensor(ns, device="cuda")][:, torch.tensor(ks, device="cuda")])
-        new = f64(mg[g][torch.tensor(ns, device="cuda")][:, torch.tensor(ks, device="cuda")])
-        for i in range(4):
-            for jj in range(4):
-                ref_w.append(orc.wgrad_entry(dyc[:, i], xc[:, jj], 0.0, False))
-                got_w.append(new[i, jj] - old[i, jj])
-    assert orc.rel_frobenius(np.array(got_w), np.array(ref_w)) <= TOL_BF16
+        rows = np.unique(np.concatenate([[a, b - 1], rng.integers(a, b, size=ROWS_PER_GROUP)]))
+        ns = rng.choice(N, size=min(COLS, N), replace=False)
+        ks = rng.choice(K, size=min(COLS, K), replace=False)
+        xr, dyr = f64(d["x"][_idx(rows)]), f64(d["dy"][_idx(rows)])
+        wr = f64(d["w"][g][_idx(ns)])            # [COLS, K]: rows n of W_g
+        wc = f64(d["w"][g][:, _idx(ks)]).T       # [COLS, N]: columns k of W_g
+        bias = f64(d["bias"][g]) if wl.bias else None
+        ref_f = np.array([[orc.fwd_entry(xr[i], wr[j], None if bias is None else bias[n])
+                           for j, n in enumerate(ns)] for i in range(len(rows))])
+        got_f = f64(y[_idx(rows)][:, _idx(ns)])
+        assert orc.rel_frobenius(got_f, ref_f) <= TOL_BF16, ("fwd", g)
+        ref_d = np.array([[orc.dgrad_entry(dyr[i], wc[j]) for j in range(len(ks))] for i in range(len(rows))])
+        got_d = f64(dx[_idx(rows)][:, _idx(ks)])
+        assert orc.rel_frobenius(got_d, ref_d) <= TOL_BF16, ("dgrad", g)
+        nw = rng.choice(N, size=WG, replace=False)
+        kw = rng.choice(K, size=WG, replace=False)
+        dyc = f64(d["dy"][a:b][:, _idx(nw)])
+        xc = f64(d["x"][a:b][:, _idx(kw)])
+        old = f64(d["main_grad"][g][_idx(nw)][:, _idx(kw)])
+        new = f64(mg[g][_idx(nw)][:, _idx(kw)])
+        ref_w = np.array([[orc.wgrad_entry(dyc[:, i], xc[:, j], old[i, j], True) for j in range(WG)]
+                          for i in range(WG)])
+        # the group's gradient (new - old) against the oracle's; old is ~1e-3
+        assert orc.rel_frobenius(new - old, ref_w - old) <= TOL_BF16, ("wgrad", g)
+        checked += 1
+    assert checked == int((m > 0).sum())
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled(name, tile_mode):
-    _sampled_parity(name)
+def test_full_size_sampled(name, pair):
+    _sampled_parity(name, pair)
     torch.cuda.empty_cache()
+
+
+# ----------------------------------------------------------------------------
+# Bounded waits: a pipeline wait that runs out is reported, and the context
+# stays usable
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("pair_", [False, True], ids=["single", "pair"])
+def test_pipeline_wait_timeout_sets_status_and_recovers(pair_):
+    """With the per-call pipeline wait bound at 1 us the first tile's
+    accumulator (64 k-blocks of loads and MMAs) cannot be ready in time: the
+    epilogue's wait runs out, GL_DEV_TIMEOUT is ORed into the status word and
+    the kernel returns (every drain of in-flight copies and MMAs keeps its own
+    bound).  The same call with the default bound then matches the oracle."""
+    G, N, K, m = 3, 512, 4096, [300, 0, 212]
+    M = sum(m)
+    d = _inputs(G, N, K, m, seed=41)
+    off, st = offsets_on_device(m, M)
+    y = sentinel_like(M, N)
+    gl.gl_fwd(d["x"], d["w"], d["bias"], off, st, y, pair=pair_, wait_limit_us=1)
+    mg = d["main_grad"].clone()
+    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True, pair=pair_, wait_limit_us=1)
+    torch.cuda.synchronize()
+    assert int(st.item()) & gl.GL_DEV_TIMEOUT
+    st.zero_()
+    gl.gl_fwd(d["x"], d["w"], d["bias"], off, st, y, pair=pair_)
+    mg = d["main_grad"].clone()
+    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True, pair=pair_)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    x64, w64, dy64 = f64(d["x"]), f64(d["w"]), f64(d["dy"])
+    assert_groups_close(f64(y), orc.fwd(x64, w64, f64(d["bias"]), m), m, what="fwd after a timeout")
+    mg0 = f64(d["main_grad"])
+    ref = orc.wgrad(x64, dy64, m, mg0, True)
+    got = f64(mg)
+    for g in range(G):
+        if m[g]:
+            assert orc.rel_frobenius(got[g] - mg0[g], ref[g] - mg0[g]) <= TOL_BF16, g
+

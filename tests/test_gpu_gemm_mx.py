@@ -19,12 +19,11 @@ from tests.gpu_util import f64, offsets_on_device, sample_rows, sentinel_like, u
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["pair", "single"])
-def tile_mode(request):
-    """Run with 256-row tiles on CTA pairs and with 128-row tiles on single CTAs."""
-    gl.gl_set_cta_pair(mxfp8=request.param == "pair")
-    yield request.param
-    gl.gl_set_cta_pair()  # defaults
+@pytest.fixture(params=[True, False], ids=["pair", "single"])
+def pair(request):
+    """256-row tiles on CTA pairs, or 128-row tiles on single CTAs (a per-call
+    option of every GEMM)."""
+    return request.param
 
 TOL_MX = 1e-2
 
@@ -66,7 +65,7 @@ SMALL = [
 
 @pytest.mark.parametrize("G,N,K,m", SMALL)
 @pytest.mark.parametrize("per_group", [False, True])
-def test_mxfp8_small(G, N, K, m, per_group, tile_mode):
+def test_mxfp8_small(G, N, K, m, per_group, pair):
     M = int(sum(m))
     d = {k: v.cuda() for k, v in synth.operands(G, M, N, K, seed=G + N + K, bias=True).items()}
     off, st = offsets_on_device(m, M, M + 32)
@@ -87,16 +86,16 @@ def test_mxfp8_small(G, N, K, m, per_group, tile_mode):
         wcs = q["w"]["scales_c"]
         bias = d["bias"]
     y = sentinel_like(M + 32, N)
-    gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], wc, ws, bias, off, st, y)
+    gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], wc, ws, bias, off, st, y, pair=pair)
     dx = sentinel_like(M + 32, K)
-    gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], wcc, wcs, off, st, dx)
+    gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], wcc, wcs, off, st, dx, pair=pair)
     mg = torch.full((G, N, K), float("nan"), device="cuda")
     mg_arg = [mg[g] for g in range(G)] if per_group else mg
     gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
-                      mg_arg, accumulate=False)
+                      mg_arg, accumulate=False, pair=pair)
     mga = d["main_grad"].clone()
     gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
-                      mga, accumulate=True)
+                      mga, accumulate=True, pair=pair)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     ref = _oracle_all(d, m, G, N, K)
@@ -116,7 +115,7 @@ def test_mxfp8_small(G, N, K, m, per_group, tile_mode):
     assert untouched(y[M:]) and untouched(dx[M:])
 
 
-def test_mxfp8_many_groups_per_group(tile_mode):
+def test_mxfp8_many_groups_per_group(pair):
     """70 groups with per-group weights and main_grad: the launches cover 64
     groups each, so the second one starts at a group whose scale k-groups
     follow those of all earlier groups."""
@@ -131,12 +130,12 @@ def test_mxfp8_many_groups_per_group(tile_mode):
     qg = [gl.group_quantize_mxfp8(d["w"][g].contiguous(), rowwise=True, colwise=True, mma_scales=True)
           for g in range(G)]
     y = gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], [t["codes_r"] for t in qg],
-                        [t["scales_r"] for t in qg], [d["bias"][g].clone() for g in range(G)], off, st)
+                        [t["scales_r"] for t in qg], [d["bias"][g].clone() for g in range(G)], off, st, pair=pair)
     dx = gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], [t["codes_c"] for t in qg],
-                           [t["scales_c"] for t in qg], off, st)
+                           [t["scales_c"] for t in qg], off, st, pair=pair)
     mg = torch.full((G, N, K), float("nan"), device="cuda")
     gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
-                      [mg[g] for g in range(G)], accumulate=False)
+                      [mg[g] for g in range(G)], accumulate=False, pair=pair)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     ref = _oracle_all(d, m, G, N, K)
@@ -152,7 +151,7 @@ def test_mxfp8_many_groups_per_group(tile_mode):
         assert orc.rel_frobenius(got_w[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad", g)
 
 
-def test_mxfp8_integer_mode_bit_exact(tile_mode):
+def test_mxfp8_integer_mode_bit_exact(pair):
     """Values in {-1,0,1}: every block scales by 2^-8 (or is all zero), the
     codes are exact, and every product sum is an exact small integer."""
     G, N, K, m = 3, 256, 128, [0, 100, 156]
@@ -161,12 +160,12 @@ def test_mxfp8_integer_mode_bit_exact(tile_mode):
     off, st = offsets_on_device(m, M)
     q = _quantize_all(d, m, G, N, K, off, st)
     y = gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], q["w"]["codes_r"].view(G, N, K),
-                        q["w"]["scales_r"], d["bias"], off, st)
+                        q["w"]["scales_r"], d["bias"], off, st, pair=pair)
     dx = gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], q["w"]["codes_c"].view(G, N, K),
-                           q["w"]["scales_c"], off, st)
+                           q["w"]["scales_c"], off, st, pair=pair)
     mg = d["main_grad"].clone()
     gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
-                      mg, accumulate=True)
+                      mg, accumulate=True, pair=pair)
     torch.cuda.synchronize()
     x64, w64, dy64 = f64(d["x"]), f64(d["w"]), f64(d["dy"])
     assert np.array_equal(synth.bf16_bits(y), orc.f64_to_bf16_rne(orc.fwd(x64, w64, f64(d["bias"]), m)))
@@ -174,55 +173,75 @@ def test_mxfp8_integer_mode_bit_exact(tile_mode):
     assert np.array_equal(f64(mg), orc.wgrad(x64, dy64, m, f64(d["main_grad"]), True))
 
 
-def test_mxfp8_full_size_sampled(tile_mode):
-    """The MXFP8 workload (G=8, K=4096, N=14336, 16384 rows in multiples of
-    128) at full size; sampled entries against the oracle, which quantizes
-    exactly the rows / columns each entry needs."""
-    wl = synth.WORKLOADS["mxfp8_g8"]
-    m = synth.m_splits_for("mxfp8_g8")
+FULL_MX = ["mxfp8_g8", "stacked_g128_uniform", "stacked_g128_ragged"]
+ROWS_PER_GROUP = 8   # random rows per group, besides the group's first and last row
+COLS = 64            # output columns sampled per group
+WG = 8               # wgrad: WG x WG sampled (n, k) entries per group
+
+
+def _idx(v):
+    return torch.as_tensor(np.asarray(v, dtype=np.int64), device="cuda")
+
+
+@pytest.mark.parametrize("name", FULL_MX)
+def test_mxfp8_full_size_sampled(name, pair):
+    """A full-size workload through the MXFP8 path: the GPU casts x, W and dy,
+    the three block-scaled GEMMs run, and every non-empty group is checked on
+    its own against the oracle, which quantizes exactly the rows / columns each
+    sampled entry needs with its own quantizer: its first, last and
+    ROWS_PER_GROUP random rows x COLS columns of y and dx, and WG x WG entries
+    of main_grad, each within 1e-2 relative Frobenius error.  The ragged
+    stacked workload keeps its unaligned split sizes, so columnwise blocks
+    restart inside 32-row blocks and groups end in partial blocks."""
+    wl = synth.WORKLOADS[name]
+    m = synth.m_splits_for(name)
     G, N, K, M = wl.G, wl.N, wl.K, wl.rows
     d = synth.operands(G, M, N, K, wl.seed, device="cuda", bias=False)
     off, st = offsets_on_device(m, M)
     q = _quantize_all(d, m, G, N, K, off, st)
     y = gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], q["w"]["codes_r"].view(G, N, K),
-                        q["w"]["scales_r"], None, off, st)
+                        q["w"]["scales_r"], None, off, st, pair=pair)
     dx = gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], q["w"]["codes_c"].view(G, N, K),
-                           q["w"]["scales_c"], off, st)
-    mg = torch.zeros(G, N, K, device="cuda")
+                           q["w"]["scales_c"], off, st, pair=pair)
+    mg = d["main_grad"].clone()
     gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st,
-                      mg, accumulate=False)
+                      mg, accumulate=True, pair=pair)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    rng = np.random.default_rng(7)
+    del q
+    rng = np.random.default_rng(wl.seed + 7)
     o = orc.offsets(m)
-    rows = sample_rows(m, 2, rng)
-    grp = np.searchsorted(o, rows, side="right") - 1
-    got_f, ref_f, got_d, ref_d = [], [], [], []
-    for r, g in zip(rows, grp):
-        r, g = int(r), int(g)
-        xr = orc.dequant_rowwise(*orc.quantize_rowwise(f64(d["x"][r:r + 1])))[0]
-        dyr = orc.dequant_rowwise(*orc.quantize_rowwise(f64(d["dy"][r:r + 1])))[0]
-        for n in rng.integers(0, N, size=6):
-            wr = orc.dequant_rowwise(*orc.quantize_rowwise(f64(d["w"][g, int(n):int(n) + 1])))[0]
-            ref_f.append(orc.fwd_entry(xr, wr, None))
-            got_f.append(float(f64(y[r, int(n):int(n) + 1])[0]))
-        for k in rng.integers(0, K, size=6):
-            col = f64(d["w"][g][:, int(k):int(k) + 1])
-            wc = orc.dequant_colwise(*orc.quantize_colwise(col, [N]), [N])[:, 0]
-            ref_d.append(orc.dgrad_entry(dyr, wc))
-            got_d.append(float(f64(dx[r, int(k):int(k) + 1])[0]))
-    assert orc.rel_frobenius(np.array(got_f), np.array(ref_f)) <= TOL_MX
-    assert orc.rel_frobenius(np.array(got_d), np.array(ref_d)) <= TOL_MX
-    got_w, ref_w = [], []
+    deq_r = lambda a: orc.dequant_rowwise(*orc.quantize_rowwise(a))
+    checked = 0
     for g in range(G):
         a, b = int(o[g]), int(o[g + 1])
         if a == b:
-            assert bool((mg[g] == 0).all())
+            assert torch.equal(mg[g], d["main_grad"][g]), ("accumulate touched an empty group", g)
             continue
-        for _ in range(6):
-            n, k = int(rng.integers(N)), int(rng.integers(K))
-            dyc = orc.dequant_colwise(*orc.quantize_colwise(f64(d["dy"][a:b, n:n + 1]), [b - a]), [b - a])[:, 0]
-            xc = orc.dequant_colwise(*orc.quantize_colwise(f64(d["x"][a:b, k:k + 1]), [b - a]), [b - a])[:, 0]
-            ref_w.append(orc.wgrad_entry(dyc, xc, 0.0, False))
-            got_w.append(float(mg[g, n, k].item()))
-    assert orc.rel_frobenius(np.array(got_w), np.array(ref_w)) <= TOL_MX
+        rows = np.unique(np.concatenate([[a, b - 1], rng.integers(a, b, size=ROWS_PER_GROUP)]))
+        ns = rng.choice(N, size=COLS, replace=False)
+        ks = rng.choice(K, size=COLS, replace=False)
+        xr = deq_r(f64(d["x"][_idx(rows)]))           # x rows, blocks along K
+        dyr = deq_r(f64(d["dy"][_idx(rows)]))         # dy rows, blocks along N
+        wr = deq_r(f64(d["w"][g][_idx(ns)]))          # W_g rows n, blocks along K
+        wcol = f64(d["w"][g][:, _idx(ks)])            # W_g columns k, blocks of 32 along N
+        wc = orc.dequant_colwise(*orc.quantize_colwise(wcol, [N]), [N]).T
+        ref_f = np.array([[orc.fwd_entry(xr[i], wr[j], None) for j in range(COLS)] for i in range(len(rows))])
+        got_f = f64(y[_idx(rows)][:, _idx(ns)])
+        assert orc.rel_frobenius(got_f, ref_f) <= TOL_MX, ("fwd", g)
+        ref_d = np.array([[orc.dgrad_entry(dyr[i], wc[j]) for j in range(COLS)] for i in range(len(rows))])
+        got_d = f64(dx[_idx(rows)][:, _idx(ks)])
+        assert orc.rel_frobenius(got_d, ref_d) <= TOL_MX, ("dgrad", g)
+        nw = rng.choice(N, size=WG, replace=False)
+        kw = rng.choice(K, size=WG, replace=False)
+        mg_g = [b - a]
+        dyc = orc.dequant_colwise(*orc.quantize_colwise(f64(d["dy"][a:b][:, _idx(nw)]), mg_g), mg_g)
+        xc = orc.dequant_colwise(*orc.quantize_colwise(f64(d["x"][a:b][:, _idx(kw)]), mg_g), mg_g)
+        old = f64(d["main_grad"][g][_idx(nw)][:, _idx(kw)])
+        new = f64(mg[g][_idx(nw)][:, _idx(kw)])
+        ref_w = np.array([[orc.wgrad_entry(dyc[:, i], xc[:, j], old[i, j], True) for j in range(WG)]
+                          for i in range(WG)])
+        assert orc.rel_frobenius(new - old, ref_w - old) <= TOL_MX, ("wgrad", g)
+        checked += 1
+    assert checked == int((m > 0).sum())
+    torch.cuda.empty_cache()

@@ -9,10 +9,13 @@ device buffer, and (the weight-cast ``noop`` use of ``grouped_linear.py``'s
 quantizers, PR #3224 "Improve device-init grouped linear module") skip a
 cast whose status word is set.
 """
+import numpy as np
 import pytest
 import torch
 
 from grouped_gemm_splits_b200 import gl, synth
+from oracle import gl_oracle as orc
+from tests.gpu_util import f64
 
 pytestmark = pytest.mark.gpu
 
@@ -94,8 +97,10 @@ def test_graph_replay_matches_eager():
 
 
 def test_graph_weight_cast_noop_flag():
-    """A captured weight cast skips its work on replays where its status word
-    (used as the noop flag) is non-zero, and runs again once it is cleared."""
+    """A captured weight cast into caller-owned (reused) buffers skips its
+    work on replays where its status word (used as the noop flag) is non-zero,
+    and once the flag is cleared writes the oracle's codes and scales into
+    those same buffers."""
     G, N, K = 2, 128, 256
     w = torch.randn(G, N, K, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).cuda()
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -117,6 +122,16 @@ def test_graph_weight_cast_noop_flag():
     flag.fill_(0)
     graph.replay()
     torch.cuda.synchronize()
+    assert int(flag.item()) == 0
+    # what the replay wrote into the reused caller buffers is the oracle's
+    # cast of W (G equal members), scales read back through the MMA layout
+    src = f64(w.reshape(G * N, K))
+    cr, sr = orc.quantize_rowwise(src)
+    cc, sc = orc.quantize_colwise(src, [N] * G)
+    assert np.array_equal(q["codes_r"].cpu().numpy().reshape(G * N, K), cr)
+    assert np.array_equal(q["scales_r"].cpu().numpy()[orc.mma_offsets_rowwise(G * N, K)], sr)
+    assert np.array_equal(q["codes_c"].cpu().numpy().reshape(G * N, K), cc)
+    assert np.array_equal(q["scales_c"].cpu().numpy()[orc.mma_offsets_colwise([N] * G, K)], sc)
     for k in ("codes_r", "codes_c"):
         assert torch.equal(q[k], first[k]), k
     del graph
