@@ -8,14 +8,17 @@ using gl::GemmCall;
 
 // Per-call GEMM options (NULL = defaults: CTA pairs, the kernels' own 2 s
 // wait bound).  False for values the header does not define.
-bool read_opts(const gl_gemm_opts* o, int* cta_pair, uint64_t* wait_ns) {
+bool read_opts(const gl_gemm_opts* o, int* cta_pair, uint64_t* wait_ns, int* hold_loads) {
   *cta_pair = 1;
   *wait_ns = 0;  // 0: the kernel's default bound
+  *hold_loads = 0;
   if (o == nullptr) return true;
   if (o->tiles != GL_TILES_PAIR && o->tiles != GL_TILES_SINGLE) return false;
   if (o->wait_limit_us > GL_WAIT_LIMIT_MAX_US) return false;
+  if (o->flags & ~GL_OPT_HOLD_LOADS) return false;
   *cta_pair = (o->tiles == GL_TILES_PAIR) ? 1 : 0;
   *wait_ns = static_cast<uint64_t>(o->wait_limit_us) * 1000u;
+  *hold_loads = (o->flags & GL_OPT_HOLD_LOADS) ? 1 : 0;
   return true;
 }
 
@@ -82,9 +85,9 @@ gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int6
                  const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  int pair = 1;
+  int pair = 1, hold = 0;
   uint64_t wait_ns = 0;
-  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
+  if (!read_opts(opts, &pair, &wait_ns, &hold)) return GL_ERR_INVALID;
   if ((x == nullptr && M > 0) || (y == nullptr && M > 0) || offsets == nullptr || status == nullptr)
     return GL_ERR_INVALID;
   if (!grouped_ok(w, G) || (bias != nullptr && !grouped_ok(*bias, G))) return GL_ERR_INVALID;
@@ -107,6 +110,7 @@ gl_status gl_fwd(const void* x, gl_grouped w, const gl_grouped* bias, const int6
   c.K = K;
   c.cta_pair = pair;
   c.wait_ns = wait_ns;
+  c.hold_loads = hold;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -115,9 +119,9 @@ gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t
                    int64_t M, int N, int K, void* dx, int64_t dx_rows, const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  int pair = 1;
+  int pair = 1, hold = 0;
   uint64_t wait_ns = 0;
-  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
+  if (!read_opts(opts, &pair, &wait_ns, &hold)) return GL_ERR_INVALID;
   if ((dy == nullptr && M > 0) || (dx == nullptr && M > 0) || offsets == nullptr || status == nullptr)
     return GL_ERR_INVALID;
   if (!grouped_ok(w, G)) return GL_ERR_INVALID;
@@ -138,6 +142,7 @@ gl_status gl_dgrad(const void* dy, gl_grouped w, const int64_t* offsets, int32_t
   c.K = K;
   c.cta_pair = pair;
   c.wait_ns = wait_ns;
+  c.hold_loads = hold;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -146,9 +151,9 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
                    int64_t M, int N, int K, gl_grouped main_grad, int accumulate, const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_gemm_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  int pair = 1;
+  int pair = 1, hold = 0;
   uint64_t wait_ns = 0;
-  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
+  if (!read_opts(opts, &pair, &wait_ns, &hold)) return GL_ERR_INVALID;
   if ((x == nullptr && M > 0) || (dy == nullptr && M > 0) || offsets == nullptr || status == nullptr)
     return GL_ERR_INVALID;
   if (!grouped_ok(main_grad, G)) return GL_ERR_INVALID;
@@ -175,6 +180,7 @@ gl_status gl_wgrad(const void* x, const void* dy, const int64_t* offsets, int32_
   c.accumulate = accumulate ? 1 : 0;
   c.cta_pair = pair;
   c.wait_ns = wait_ns;
+  c.hold_loads = hold;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm(c);
 }
@@ -196,9 +202,9 @@ gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_group
                        const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_mx_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  int pair = 1;
+  int pair = 1, hold = 0;
   uint64_t wait_ns = 0;
-  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
+  if (!read_opts(opts, &pair, &wait_ns, &hold)) return GL_ERR_INVALID;
   if (((x_codes == nullptr || x_scales == nullptr || y == nullptr) && M > 0) || offsets == nullptr ||
       status == nullptr)
     return GL_ERR_INVALID;
@@ -226,6 +232,7 @@ gl_status gl_fwd_mxfp8(const uint8_t* x_codes, const uint8_t* x_scales, gl_group
   c.K = K;
   c.cta_pair = pair;
   c.wait_ns = wait_ns;
+  c.hold_loads = hold;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
@@ -235,9 +242,9 @@ gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_g
                          int64_t M, int N, int K, void* dx, int64_t dx_rows, const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_mx_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  int pair = 1;
+  int pair = 1, hold = 0;
   uint64_t wait_ns = 0;
-  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
+  if (!read_opts(opts, &pair, &wait_ns, &hold)) return GL_ERR_INVALID;
   if (((dy_codes == nullptr || dy_scales == nullptr || dx == nullptr) && M > 0) || offsets == nullptr ||
       status == nullptr)
     return GL_ERR_INVALID;
@@ -263,6 +270,7 @@ gl_status gl_dgrad_mxfp8(const uint8_t* dy_codes, const uint8_t* dy_scales, gl_g
   c.K = K;
   c.cta_pair = pair;
   c.wait_ns = wait_ns;
+  c.hold_loads = hold;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }
@@ -272,9 +280,9 @@ gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, co
                          int64_t M, int N, int K, gl_grouped main_grad, int accumulate, const gl_gemm_opts* opts, void* stream) {
   gl_status st = check_mx_dims(G, M, N, K);
   if (st != GL_OK) return st;
-  int pair = 1;
+  int pair = 1, hold = 0;
   uint64_t wait_ns = 0;
-  if (!read_opts(opts, &pair, &wait_ns)) return GL_ERR_INVALID;
+  if (!read_opts(opts, &pair, &wait_ns, &hold)) return GL_ERR_INVALID;
   if (((x_codes_c == nullptr || x_scales_c == nullptr || dy_codes_c == nullptr || dy_scales_c == nullptr) &&
        M > 0) ||
       offsets == nullptr || status == nullptr)
@@ -304,6 +312,7 @@ gl_status gl_wgrad_mxfp8(const uint8_t* x_codes_c, const uint8_t* x_scales_c, co
   c.accumulate = accumulate ? 1 : 0;
   c.cta_pair = pair;
   c.wait_ns = wait_ns;
+  c.hold_loads = hold;
   c.stream = to_stream(stream);
   return gl::launch_grouped_gemm_mx(c);
 }

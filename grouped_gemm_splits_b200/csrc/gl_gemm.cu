@@ -39,7 +39,7 @@
 namespace gl {
 namespace {
 
-constexpr int BK = 64;  // contraction elements per stage (one 128-byte swizzle row)
+constexpr int BK = 64;  // contraction elements of a K-major stage (one 128-byte swizzle row)
 constexpr int kPG = 64;  // per-group tensor maps carried by one launch
 constexpr int kSmemBudget = 212992;  // 6 stages of 32 KB + (wgrad) 16 KB of epilogue transposes
 constexpr int kBand = 8;  // tile rows per rasterisation band
@@ -49,8 +49,12 @@ struct Cfg {
   static constexpr int kTileM = 128 * CG;          // accumulator rows per tile (pair)
   static constexpr int kTileN = 256;               // accumulator columns
   static constexpr int kBRows = kTileN / CG;       // rows of the B operand held per CTA
-  static constexpr int kABytes = 128 * BK * 2;     // 16 KB
-  static constexpr int kBBytes = kBRows * BK * 2;  // 32 KB (CG 1) or 16 KB (CG 2)
+  // contraction elements per stage; only wgrad, whose operands are both
+  // MN-major, could take longer stages (a K-major box spans one 128-byte row)
+  static constexpr int kBK = BK;
+  static constexpr int kMNChunk = 128 * kBK;        // bytes of a 64-column MN-major chunk of a stage
+  static constexpr int kABytes = 128 * kBK * 2;     // 16 KB
+  static constexpr int kBBytes = kBRows * kBK * 2;  // 32 KB (CG 1) or 16 KB (CG 2)
   static constexpr int kStageBytes = kABytes + kBBytes;
   // epilogue warps, one per TMEM lane quarter (eight for wgrad measured no
   // faster and cost a pipeline stage of staging space)
@@ -86,6 +90,7 @@ struct GemmParams {
   int has_bias;
   int accumulate;
   uint64_t wait_ns;  // bound on each pipeline wait
+  int hold_loads;    // testing: the producer issues no loads
 };
 
 template <bool PG>
@@ -158,7 +163,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const Gemm
   if (MODE == kWgrad) {
     tl.r0 = o0;
     tl.r1 = o0 + m;
-    tl.num_kb = ceil_div_i(m, BK);
+    tl.num_kb = ceil_div_i(m, C::kBK);
   } else {
     tl.r0 = o0 + static_cast<int64_t>(tl.mt) * C::kTileM;
     tl.r1 = o0 + m;
@@ -179,9 +184,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Zero rows [r_from, r_to) of this CTA's A and B stage buffers (MN-major, 64
-// rows x 128 bytes per 8 KB chunk) so rows past a group's end add nothing to
-// a wgrad contraction.  Executed by one full warp.
+// Zero rows [r_from, r_to) of this CTA's A and B stage buffers (MN-major,
+// kBK rows x 128 bytes per chunk of 64 columns) so rows past a group's end
+// add nothing to a wgrad contraction.  Executed by one full warp.
 template <int MODE, int CG>
 __device__ __forceinline__ void zero_tail_rows(uint8_t* sa, uint8_t* sb, int r_from, int r_to, int lane) {
   using C = Cfg<MODE, CG>;
@@ -193,7 +198,7 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* sa, uint8_t* sb, int r_f
     const int chunk = idx / per_chunk;
     const int rem = idx - chunk * per_chunk;
     const int row = r_from + (rem >> 3);
-    uint8_t* base = (chunk < kChunksA) ? (sa + chunk * 8192) : (sb + (chunk - kChunksA) * 8192);
+    uint8_t* base = (chunk < kChunksA) ? (sa + chunk * C::kMNChunk) : (sb + (chunk - kChunksA) * C::kMNChunk);
     *reinterpret_cast<uint4*>(base + row * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
@@ -303,6 +308,10 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
         const Tile tl = decode_tile<MODE, CG>(t, prefix, p);
         for (int kb = 0; kb < tl.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.wait_ns)) { report_abort(abort_flag, p.status); break; }
+          if (p.hold_loads) {  // testing the timeout path: this stage never lands
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            continue;
+          }
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
@@ -316,20 +325,20 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
             tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0 + hr));
 #pragma unroll
             for (int c = 0; c < C::kBRows / 64; ++c) {
-              if (PG) tma_load_2d(sb + c * 8192, pg.map(tl.g), &full[stage], n0 + c * 64, kb * BK);
-              else    tma_load_3d(sb + c * 8192, &p.tmB, &full[stage], n0 + c * 64, kb * BK, tl.g);
+              if (PG) tma_load_2d(sb + c * C::kMNChunk, pg.map(tl.g), &full[stage], n0 + c * 64, kb * BK);
+              else    tma_load_3d(sb + c * C::kMNChunk, &p.tmB, &full[stage], n0 + c * 64, kb * BK, tl.g);
             }
           } else {
             // operand strips are read again by the neighbouring tiles of the
             // band: keep them in L2 ahead of the streamed main_grad lines
-            const int32_t row = static_cast<int32_t>(tl.r0 + kb * BK);
+            const int32_t row = static_cast<int32_t>(tl.r0 + kb * C::kBK);
             const int m0 = tl.mt * C::kTileM + hr;
             const int n0 = tl.nt * C::kTileN + hb;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) tma_load_2d_hint(sa + c * 8192, &p.tmA, &full[stage], m0 + c * 64, row, keep);
+            for (int c = 0; c < 2; ++c) tma_load_2d_hint(sa + c * C::kMNChunk, &p.tmA, &full[stage], m0 + c * 64, row, keep);
 #pragma unroll
             for (int c = 0; c < C::kBRows / 64; ++c)
-              tma_load_2d_hint(sb + c * 8192, &p.tmB, &full[stage], n0 + c * 64, row, keep);
+              tma_load_2d_hint(sb + c * C::kMNChunk, &p.tmB, &full[stage], n0 + c * 64, row, keep);
           }
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -370,7 +379,7 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
           // On a ragged wgrad tail the peer zeroes rows of its stage before
           // relaying; acquire at cluster scope so those writes are visible.
           const bool peer_zeroed = CG == 2 && MODE == kWgrad && kb == tl.num_kb - 1 &&
-                                   static_cast<int>(tl.r1 - tl.r0) - kb * BK < BK;
+                                   static_cast<int>(tl.r1 - tl.r0) - kb * C::kBK < C::kBK;
           const bool landed = peer_zeroed ? mbar_wait_acq_cluster(&full[stage], phase, abort_flag, p.wait_ns)
                                           : mbar_wait(&full[stage], phase, abort_flag, p.wait_ns);
           if (!__all_sync(0xffffffffu, landed)) {
@@ -381,12 +390,12 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
           tc_fence_after();
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
-          int ksteps = BK / 16;
+          int ksteps = C::kBK / 16;
           if (MODE == kWgrad && kb == tl.num_kb - 1) {
             // Ragged contraction: skip whole 16-row MMA steps past the group's
             // end and zero the rows of the last partial step.
-            const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
-            if (valid < BK) {
+            const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * C::kBK;
+            if (valid < C::kBK) {
               ksteps = (valid + 15) >> 4;
               zero_tail_rows<MODE, CG>(sa, sb, valid, ksteps * 16, lane);
             }
@@ -395,9 +404,9 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
           if (lane == 0) {
             const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
             for (int ks = 0; ks < ksteps; ++ks) {
-              const uint64_t ad = C::kAMN ? smem_desc_sw128(a0 + ks * 2048, 8192, 1024)
+              const uint64_t ad = C::kAMN ? smem_desc_sw128(a0 + ks * 2048, C::kMNChunk, 1024)
                                           : smem_desc_sw128(a0 + ks * 32, 16, 1024);
-              const uint64_t bd = C::kBMN ? smem_desc_sw128(b0 + ks * 2048, 8192, 1024)
+              const uint64_t bd = C::kBMN ? smem_desc_sw128(b0 + ks * 2048, C::kMNChunk, 1024)
                                           : smem_desc_sw128(b0 + ks * 32, 16, 1024);
               const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
               if (CG == 2) mma_bf16_ss_pair(d_tmem, ad, bd, C::kIdesc, acc);
@@ -415,7 +424,7 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
           if (tl.num_kb > 0) {
             if (CG == 2) tc_commit_pair_mc(&tfull[buf], 0x3);
             else         tc_commit(&tfull[buf]);
-          } else {
+          } else if (!p.hold_loads) {
             // nothing accumulated: the epilogues write zeros
             mbar_arrive(&tfull[buf]);
             if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&tfull[buf]), 1));
@@ -444,8 +453,8 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
           }
           bool zeroed = false;
           if (MODE == kWgrad && kb == tl.num_kb - 1) {
-            const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * BK;
-            if (valid < BK) {
+            const int valid = static_cast<int>(tl.r1 - tl.r0) - kb * C::kBK;
+            if (valid < C::kBK) {
               uint8_t* sa = smem + stage * C::kStageBytes;
               zero_tail_rows<MODE, CG>(sa, sa + C::kABytes, valid, ((valid + 15) >> 4) * 16, lane);
               zeroed = true;
@@ -700,6 +709,7 @@ gl_status launch_mode(const GemmCall& c) {
   prm.K = c.K;
   prm.accumulate = c.accumulate;
   prm.wait_ns = c.wait_ns ? c.wait_ns : kWaitLimitNs;
+  prm.hold_loads = c.hold_loads;
   prm.has_bias = (MODE == kFwd && c.bias != nullptr) ? 1 : 0;
   const uint64_t Mrows = c.M > 0 ? static_cast<uint64_t>(c.M) : 1;  // a map needs >= 1 row
   bool ok = true;
@@ -708,8 +718,8 @@ gl_status launch_mode(const GemmCall& c) {
   } else if (MODE == kDgrad) {
     ok &= make_2d(&prm.tmA, c.a, c.N, Mrows, BK, 128, BF, 2);
   } else {
-    ok &= make_2d(&prm.tmA, c.a, c.N, Mrows, 64, BK, BF, 2);
-    ok &= make_2d(&prm.tmB, c.b, c.K, Mrows, 64, BK, BF, 2);
+    ok &= make_2d(&prm.tmA, c.a, c.N, Mrows, 64, Cf::kBK, BF, 2);
+    ok &= make_2d(&prm.tmB, c.b, c.K, Mrows, 64, Cf::kBK, BF, 2);
   }
   if (!ok) return GL_ERR_UNSUPPORTED;
 

@@ -7,17 +7,16 @@
 // columnwise for wgrad), computed as sum_k (q_a 2^sa)(q_b 2^sb) by
 // tcgen05.mma kind::mxf8f6f4.block_scale with fp32 accumulation in TMEM.
 //
-// Output tile 128*CG x TN.  With CG = 2 a cluster pair shares the tile
-// (tcgen05 cta_group::2): each CTA loads its own 128 rows of A and TN/2 rows
+// Output tile 128*CG x 256.  With CG = 2 a cluster pair shares the tile
+// (tcgen05 cta_group::2): each CTA loads its own 128 rows of A and 128 rows
 // of B; the peer relays "stage landed" to the leader, which issues the MMAs.
-// fprop / dgrad: TN = 256 and one fp32 accumulator (256 TMEM columns); eight
-// epilogue warps copy it to registers and free it at once, so the next tile's
-// MMAs overlap the stores.  wgrad: TN = 192 and two accumulators (384
-// columns); eight epilogue warps (half the columns each) transpose 32 x 32
-// fp32 chunks through shared memory and add them into main_grad with
-// coalesced 16-byte vector reductions (each tile's main_grad rows first
-// pulled into L2 with bulk prefetches).  The remaining TMEM columns hold the
-// scale-factor slots.
+// One fp32 accumulator (256 TMEM columns) per tile: eight epilogue warps (two
+// per TMEM lane quarter, 128 columns each) copy it to registers and free it
+// at once, so the next tile's MMAs overlap the stores -- fprop / dgrad round
+// to bf16 (+ bias); wgrad transposes 32 x 32 fp32 chunks through shared
+// memory and adds them into main_grad with coalesced 16-byte vector
+// reductions (each tile's main_grad rows first pulled into L2 with bulk
+// prefetches).  The remaining TMEM columns hold the scale-factor slots.
 //
 // Per stage (128 contraction elements = four MMAs of K=32) the producer
 // TMA-loads the codes (128-byte swizzle) and the scales.  The scales arrive
@@ -27,12 +26,9 @@
 // one atom for the CTA's 128 A rows and two consecutive atoms (256 rows)
 // covering the tile's B rows.  The MMA thread copies them to TMEM with
 // tcgen05.cp.32x128b.warpx4 and selects scale byte kb of each MMA through the
-// instruction descriptor.  B row i of a tile that starts at operand row
-// 128c + 32s reads TMEM column (slot + s) + i/32, so the MMA's scale address is
-// offset by s columns: 0 for 256-row tiles, 0 or 2 for 192-row tiles (their
-// starts are multiples of 64 rows).  A tiles (fprop / dgrad) start on 128-row boundaries of
-// the packed activations: a group's first tile may begin inside the previous
-// group, and only the group's own rows are stored.
+// instruction descriptor.  A tiles (fprop / dgrad) start on 128-row
+// boundaries of the packed activations: a group's first tile may begin inside
+// the previous group, and only the group's own rows are stored.
 //
 // The only generic shared-memory writes on the main loop are the zeroed rows
 // of a ragged wgrad contraction tail (once per tile); on a pair the peer
@@ -56,14 +52,14 @@ constexpr int kBand = 8;
 constexpr int kSfSlots = 4;      // slot j: A at +0 (4 columns), B at +4 (8 columns)
 constexpr int kSfSlotCols = 16;
 constexpr int kSfABytes = 512;   // one atom
-constexpr int kAtomsB = 2;       // 256 B rows: a whole 256-row tile, or a 192-row tile 0 or 64 rows in
+constexpr int kAtomsB = 2;       // the 256 B rows of a tile
 constexpr int kSfBytes = 2048;   // A atom + B atoms, padded to keep stages 1 KB aligned
 static_assert(kSfABytes + kAtomsB * 512 <= kSfBytes, "scale staging");
 
 template <int MODE, int CG>
 struct CfgMX {
-  static constexpr int kTN = (MODE == kWgrad) ? 192 : 256;  // accumulator columns
-  static constexpr int kAccBufs = (MODE == kWgrad) ? 2 : 1;
+  static constexpr int kTN = 256;     // accumulator columns
+  static constexpr int kAccBufs = 1;  // drained to registers at once, so the next tile's MMAs overlap the stores
   static constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, half the columns each
   static constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, 1 MMA / relay, then epilogue
   static constexpr int kSfCol0 = kAccBufs * kTN;        // first TMEM column of the scale-factor slots
@@ -74,8 +70,7 @@ struct CfgMX {
   static constexpr int kBChunks = (kBRows + 127) / 128;
   static constexpr int kBAlloc = (MODE == kFwd) ? kBRows * BK : kBChunks * 128 * BK;
   static constexpr int kBLoad = kBAlloc;
-  static_assert((kTN % 128 == 0 ? 0 : 64) + kTN <= 128 * kAtomsB && kTN % 64 == 0,
-                "B tile must stay inside the loaded scale atoms");
+  static_assert(kTN == 128 * kAtomsB, "a B tile is exactly the loaded scale atoms");
   static constexpr int kStageBytes = kABytes + kBAlloc + kSfBytes;  // 50 KB (CG 1) / 34 KB (CG 2)
   static constexpr int kStagingBytes = (MODE == kWgrad) ? kEpiWarps * 32 * 32 * 4 : 0;  // one 4 KB transpose per epilogue warp
   static constexpr int kStages = CG == 2 ? ((MODE == kWgrad) ? 5 : 6) : ((MODE == kWgrad) ? 3 : 4);
@@ -111,6 +106,7 @@ struct MxParams {
   int has_bias;
   int accumulate;
   uint64_t wait_ns;  // bound on each pipeline wait
+  int hold_loads;    // testing: the producer issues no loads
 };
 
 template <bool PG>
@@ -350,6 +346,10 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
         const int n0 = tl.nt * TN;  // first B operand row of the tile
         for (int kb = 0; kb < tl.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.wait_ns)) { report_abort(abort_flag, p.status); break; }
+          if (p.hold_loads) {  // testing the timeout path: this stage never lands
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            continue;
+          }
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           uint8_t* sf = sb + C::kBAlloc;
@@ -423,8 +423,6 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * TN;
-        // the tile's first B row sits 32 * sh rows into the first loaded atom
-        const uint32_t sh = static_cast<uint32_t>((tl.nt * TN) & 127) >> 5;
         bool ok = true;
         for (int kb = 0; kb < tl.num_kb; ++kb, ++kiter) {
           int ksteps = BK / 32;
@@ -462,7 +460,7 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
 #pragma unroll
               for (int a = 0; a < kAtomsB; ++a) tmem_cp_32x128b_x4(sfb0 + 4 * a, smem_desc_sf(pb + 512 * a));
             }
-            const uint32_t sfb = sfb0 + sh;
+            const uint32_t sfb = sfb0;
             const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
             for (int ks = 0; ks < ksteps; ++ks) {
               const uint64_t ad = C::kAMN ? smem_desc_sw128(a0 + ks * 4096, 16384, 1024)
@@ -485,7 +483,7 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
           if (tl.num_kb > 0) {
             if (CG == 2) tc_commit_pair_mc(&tfull[buf], 0x3);
             else         tc_commit(&tfull[buf]);
-          } else {
+          } else if (!p.hold_loads) {  // nothing accumulated: the epilogues write zeros
             mbar_arrive(&tfull[buf]);
             if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&tfull[buf]), 1));
           }
@@ -617,51 +615,59 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
           }
         }
       } else {
-        // main_grad rows n0 + 0..31 (this warp's TMEM lanes) x columns k0 + 32c..:
-        // each [32 x 32] fp32 chunk goes through a 4 KB per-warp shared-memory
-        // transpose (16-byte pieces, XOR-swizzled: conflict-free both ways), so
-        // that 8 lanes cover one row's 128 contiguous bytes, then leaves as
-        // coalesced 16-byte vector reductions (accumulate) or stores
+        // main_grad rows n0 + 0..31 (this warp's TMEM lanes) x columns k0 .. k0+127
+        // (its half of the tile): copy them to registers and free the
+        // accumulator, so the next tile's MMAs run while these sums leave.
+        // Each [32 x 32] fp32 chunk then goes through a 4 KB per-warp
+        // shared-memory transpose (16-byte pieces, XOR-swizzled: conflict-free
+        // both ways), so that 8 lanes cover one row's 128 contiguous bytes, and
+        // leaves as coalesced 16-byte vector reductions (accumulate) or stores
         // (overwrite): full-line transactions, many in flight, no waits.
         float* stg = reinterpret_cast<float*>(smem + C::kStagingOffset) + (warp - 2) * (32 * 32);
         constexpr int kCols = TN / 2;  // columns of this warp (its half)
+        constexpr int kChunks = kCols / 32;
         const int n0 = tl.mt * TMt + hr + q * 32;
         const int k0 = tl.nt * TN + h * kCols;
-        const int nchunks = max(0, min(kCols / 32, cdiv(p.K - k0, 32)));
-        const bool have_acc = tl.num_kb > 0;
-        float* gbase = PG ? pg.m(tl.g) : p.mg + static_cast<int64_t>(tl.g) * p.N * p.K;
-        const int sub = lane >> 3, piece = lane & 7;  // read side: row 4i + sub, 16-byte piece
-        for (int c = 0; c < nchunks; ++c) {
-          uint32_t r[32];
-          if (have_acc) {
-            tmem_ld_32x32b_x32(tacc + h * kCols + c * 32, r);
-            tmem_ld_wait();
-            tmem_reg_fence(r);
-          } else {
+        const bool in_k = k0 < p.K;  // K % 128 == 0: the half is all inside K or all past it
+        uint32_t r[kChunks][32];
+        if (tl.num_kb > 0 && in_k) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = 0u;
-          }
-          if (c == nchunks - 1) release_acc();
+          for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(tacc + h * kCols + c * 32, r[c]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) tmem_reg_fence(r[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[c][j] = 0u;  // an empty group's overwrite: zeros
+        }
+        release_acc();
+        if (in_k) {
+          float* gbase = PG ? pg.m(tl.g) : p.mg + static_cast<int64_t>(tl.g) * p.N * p.K;
+          const int sub = lane >> 3, piece = lane & 7;  // read side: row 4i + sub, 16-byte piece
           float* mine = stg + lane * 32;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(mine + ((j ^ (lane & 7)) << 2)) =
-                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-          __syncwarp();
-          const int col = k0 + c * 32 + piece * 4;
+          for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int row = 4 * i + sub;
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + row * 32 + ((piece ^ (row & 7)) << 2));
-            if (n0 + row < p.N && col < p.K) {  // K % 128 == 0: four columns are all in or all out
-              float* dst = gbase + static_cast<int64_t>(n0 + row) * p.K + col;
-              if (p.accumulate) red_add_v4(dst, v.x, v.y, v.z, v.w);
-              else *reinterpret_cast<uint4*>(dst) = v;
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(mine + ((j ^ (lane & 7)) << 2)) =
+                  make_uint4(r[c][4 * j], r[c][4 * j + 1], r[c][4 * j + 2], r[c][4 * j + 3]);
+            __syncwarp();
+            const int col = k0 + c * 32 + piece * 4;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int row = 4 * i + sub;
+              const uint4 v = *reinterpret_cast<const uint4*>(stg + row * 32 + ((piece ^ (row & 7)) << 2));
+              if (n0 + row < p.N) {
+                float* dst = gbase + static_cast<int64_t>(n0 + row) * p.K + col;
+                if (p.accumulate) red_add_v4(dst, v.x, v.y, v.z, v.w);
+                else *reinterpret_cast<uint4*>(dst) = v;
+              }
             }
+            __syncwarp();  // the next chunk overwrites the transpose buffer
           }
-          __syncwarp();  // the next chunk overwrites the transpose buffer
         }
-        if (nchunks == 0) release_acc();  // this warp's half lies past K: nothing to read
       }
     }
   }
@@ -779,6 +785,7 @@ gl_status mx_mode(const MxCall& c) {
   prm.K = c.K;
   prm.accumulate = c.accumulate;
   prm.wait_ns = c.wait_ns ? c.wait_ns : kWaitLimitNs;
+  prm.hold_loads = c.hold_loads;
   prm.has_bias = (MODE == kFwd && c.bias != nullptr) ? 1 : 0;
   prm.offsets_all = c.offsets;
   const uint64_t M = c.M > 0 ? static_cast<uint64_t>(c.M) : 1;

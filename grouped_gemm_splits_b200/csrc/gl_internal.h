@@ -41,6 +41,7 @@ struct GemmCall {
   int accumulate;
   int cta_pair;  // 1: 256x256 tiles on CTA pairs (cta_group::2); 0: 128x256 tiles per CTA
   uint64_t wait_ns;  // bound on each pipeline wait inside the kernel
+  int hold_loads;    // testing: issue no loads (every pipeline wait runs out)
   cudaStream_t stream;
 };
 
@@ -65,8 +66,9 @@ struct MxCall {
   int64_t M;
   int N, K;
   int accumulate;
-  int cta_pair;  // 1: CTA pairs (256x256 fprop/dgrad, 256x192 wgrad tiles); 0: single CTAs (128x256 / 128x192)
+  int cta_pair;  // 1: 256x256 tiles on CTA pairs; 0: 128x256 tiles on single CTAs
   uint64_t wait_ns;  // bound on each pipeline wait inside the kernel
+  int hold_loads;    // testing: issue no loads (every pipeline wait runs out)
   cudaStream_t stream;
 };
 

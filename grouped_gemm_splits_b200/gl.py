@@ -36,8 +36,11 @@ class GlGrouped(ctypes.Structure):
 GL_TILES_PAIR, GL_TILES_SINGLE = 0, 1
 
 
+GL_OPT_HOLD_LOADS = 1
+
+
 class GlGemmOpts(ctypes.Structure):
-    _fields_ = [("tiles", ctypes.c_int), ("wait_limit_us", ctypes.c_uint32)]
+    _fields_ = [("tiles", ctypes.c_int), ("wait_limit_us", ctypes.c_uint32), ("flags", ctypes.c_uint32)]
 
 
 class GlError(RuntimeError):
@@ -124,11 +127,11 @@ def _shape_nk(w: TensorOrList):
     return tuple((w if isinstance(w, torch.Tensor) else w[0]).shape[-2:])
 
 
-def _opts(pair: bool, wait_limit_us: int):
+def _opts(pair: bool, wait_limit_us: int, flags: int = 0):
     """Per-call GEMM options (``gl_gemm_opts``); None for the defaults."""
-    if pair and not wait_limit_us:
+    if pair and not wait_limit_us and not flags:
         return None
-    return ctypes.pointer(GlGemmOpts(GL_TILES_PAIR if pair else GL_TILES_SINGLE, wait_limit_us))
+    return ctypes.pointer(GlGemmOpts(GL_TILES_PAIR if pair else GL_TILES_SINGLE, wait_limit_us, flags))
 
 
 def gl_offsets(m_splits: torch.Tensor, expect_rows: int, out_rows: Optional[int] = None,
@@ -147,7 +150,7 @@ def gl_offsets(m_splits: torch.Tensor, expect_rows: int, out_rows: Optional[int]
 
 
 def gl_fwd(x: torch.Tensor, w: TensorOrList, bias: Optional[TensorOrList], offsets: torch.Tensor,
-           status: torch.Tensor, y: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0) -> torch.Tensor:
+           status: torch.Tensor, y: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0, opt_flags: int = 0) -> torch.Tensor:
     """y rows of group g = x rows of group g @ W_g^T (+ b_g).  ``y`` may be a
     caller buffer with more rows than x; only the valid rows are written."""
     G = offsets.numel() - 1
@@ -163,13 +166,13 @@ def gl_fwd(x: torch.Tensor, w: TensorOrList, bias: Optional[TensorOrList], offse
         bg, keep_b = _grouped(bias, G)
         bptr = ctypes.pointer(bg)
     _check(load().gl_fwd(x.data_ptr(), wg, bptr, offsets.data_ptr(), status.data_ptr(), G, M, N, K,
-                         y.data_ptr(), y.shape[0], _opts(pair, wait_limit_us), _stream()), "gl_fwd")
+                         y.data_ptr(), y.shape[0], _opts(pair, wait_limit_us, opt_flags), _stream()), "gl_fwd")
     del keep_w, keep_b
     return y
 
 
 def gl_dgrad(dy: torch.Tensor, w: TensorOrList, offsets: torch.Tensor, status: torch.Tensor,
-             dx: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0) -> torch.Tensor:
+             dx: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0, opt_flags: int = 0) -> torch.Tensor:
     """dx rows of group g = dy rows of group g @ W_g."""
     G = offsets.numel() - 1
     M, N = dy.shape
@@ -179,20 +182,20 @@ def gl_dgrad(dy: torch.Tensor, w: TensorOrList, offsets: torch.Tensor, status: t
         dx = torch.empty(M, K, dtype=torch.bfloat16, device=dy.device)
     wg, keep_w = _grouped(w, G)
     _check(load().gl_dgrad(dy.data_ptr(), wg, offsets.data_ptr(), status.data_ptr(), G, M, N, K,
-                           dx.data_ptr(), dx.shape[0], _opts(pair, wait_limit_us), _stream()), "gl_dgrad")
+                           dx.data_ptr(), dx.shape[0], _opts(pair, wait_limit_us, opt_flags), _stream()), "gl_dgrad")
     del keep_w
     return dx
 
 
 def gl_wgrad(x: torch.Tensor, dy: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
-             main_grad: TensorOrList, accumulate: bool = True, pair: bool = True, wait_limit_us: int = 0) -> TensorOrList:
+             main_grad: TensorOrList, accumulate: bool = True, pair: bool = True, wait_limit_us: int = 0, opt_flags: int = 0) -> TensorOrList:
     """main_grad[g] (+)= dy_g^T @ x_g (fp32)."""
     G = offsets.numel() - 1
     M, K = x.shape
     N = dy.shape[1]
     mg, keep = _grouped(main_grad, G)
     _check(load().gl_wgrad(x.data_ptr(), dy.data_ptr(), offsets.data_ptr(), status.data_ptr(), G,
-                           M, N, K, mg, 1 if accumulate else 0, _opts(pair, wait_limit_us), _stream()), "gl_wgrad")
+                           M, N, K, mg, 1 if accumulate else 0, _opts(pair, wait_limit_us, opt_flags), _stream()), "gl_wgrad")
     del keep
     return main_grad
 
@@ -330,7 +333,7 @@ def _grouped_any(t: TensorOrList, G: int):
 
 def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorOrList, w_scales: TensorOrList,
                  bias: Optional[TensorOrList], offsets: torch.Tensor, status: torch.Tensor,
-                 y: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0) -> torch.Tensor:
+                 y: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0, opt_flags: int = 0) -> torch.Tensor:
     """fprop on MXFP8 operands: x rowwise codes [M,K] + scale atoms; W rowwise
     codes [G,N,K] (or G x [N,K]) + scale atoms (all scales ``mma_scales``)."""
     G = offsets.numel() - 1
@@ -345,7 +348,7 @@ def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorO
         bg, k3 = _grouped(bias, G)
         bptr = ctypes.pointer(bg)
     _check(load().gl_fwd_mxfp8(x_codes.data_ptr(), x_scales.data_ptr(), wc, ws, bptr, offsets.data_ptr(),
-                               status.data_ptr(), G, M, N, K, y.data_ptr(), y.shape[0], _opts(pair, wait_limit_us), _stream()),
+                               status.data_ptr(), G, M, N, K, y.data_ptr(), y.shape[0], _opts(pair, wait_limit_us, opt_flags), _stream()),
            "gl_fwd_mxfp8")
     del k1, k2, k3
     return y
@@ -353,7 +356,7 @@ def gl_fwd_mxfp8(x_codes: torch.Tensor, x_scales: torch.Tensor, w_codes: TensorO
 
 def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: TensorOrList,
                    w_scales_c: TensorOrList, offsets: torch.Tensor, status: torch.Tensor,
-                   dx: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0) -> torch.Tensor:
+                   dx: Optional[torch.Tensor] = None, pair: bool = True, wait_limit_us: int = 0, opt_flags: int = 0) -> torch.Tensor:
     """dgrad on MXFP8 operands: dy rowwise codes [M,N] + scale atoms; W
     columnwise codes [G,N,K] + columnwise scale atoms."""
     G = offsets.numel() - 1
@@ -364,7 +367,7 @@ def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: T
     wc, k1 = _grouped_any(w_codes_c, G)
     ws, k2 = _grouped_any(w_scales_c, G)
     _check(load().gl_dgrad_mxfp8(dy_codes.data_ptr(), dy_scales.data_ptr(), wc, ws, offsets.data_ptr(),
-                                 status.data_ptr(), G, M, N, K, dx.data_ptr(), dx.shape[0], _opts(pair, wait_limit_us), _stream()),
+                                 status.data_ptr(), G, M, N, K, dx.data_ptr(), dx.shape[0], _opts(pair, wait_limit_us, opt_flags), _stream()),
            "gl_dgrad_mxfp8")
     del k1, k2
     return dx
@@ -372,7 +375,7 @@ def gl_dgrad_mxfp8(dy_codes: torch.Tensor, dy_scales: torch.Tensor, w_codes_c: T
 
 def gl_wgrad_mxfp8(x_codes_c: torch.Tensor, x_scales_c: torch.Tensor, dy_codes_c: torch.Tensor,
                    dy_scales_c: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
-                   main_grad: TensorOrList, accumulate: bool = True, pair: bool = True, wait_limit_us: int = 0) -> TensorOrList:
+                   main_grad: TensorOrList, accumulate: bool = True, pair: bool = True, wait_limit_us: int = 0, opt_flags: int = 0) -> TensorOrList:
     """wgrad on MXFP8 operands: x and dy columnwise codes + columnwise scale atoms."""
     G = offsets.numel() - 1
     M, K = x_codes_c.shape
@@ -380,6 +383,6 @@ def gl_wgrad_mxfp8(x_codes_c: torch.Tensor, x_scales_c: torch.Tensor, dy_codes_c
     mg, keep = _grouped(main_grad, G)
     _check(load().gl_wgrad_mxfp8(x_codes_c.data_ptr(), x_scales_c.data_ptr(), dy_codes_c.data_ptr(),
                                  dy_scales_c.data_ptr(), offsets.data_ptr(), status.data_ptr(), G, M, N, K, mg,
-                                 1 if accumulate else 0, _opts(pair, wait_limit_us), _stream()), "gl_wgrad_mxfp8")
+                                 1 if accumulate else 0, _opts(pair, wait_limit_us, opt_flags), _stream()), "gl_wgrad_mxfp8")
     del keep
     return main_grad

@@ -89,27 +89,33 @@ const char* gl_status_string(gl_status s);
  * They belong to the one call: the library keeps no mode between calls, so
  * callers on different threads never change each other's kernels.
  *
- *   tiles          GL_TILES_PAIR (0, the default): 256-row output tiles on
- *                  pairs of CTAs (tcgen05 cta_group::2, one CTA per SM) --
- *                  bf16 256 x 256; MXFP8 256 x 256 (fprop, dgrad) and
- *                  256 x 192 (wgrad).  GL_TILES_SINGLE: 128-row tiles on
- *                  single CTAs (bf16 128 x 256; MXFP8 128 x 256 and
- *                  128 x 192).  Results agree within rounding.
+ *   tiles          GL_TILES_PAIR (0, the default): 256 x 256 output tiles
+ *                  on pairs of CTAs (tcgen05 cta_group::2, one CTA per SM).
+ *                  GL_TILES_SINGLE: 128 x 256 tiles on single CTAs.  Results
+ *                  agree within rounding.
  *   wait_limit_us  bound, in microseconds, on each wait of the kernel's
- *                  load -> MMA -> epilogue pipeline; 0 = the default (2 s),
- *                  at most GL_WAIT_LIMIT_MAX_US.  A wait that runs out ORs
+ *                  load -> MMA -> epilogue pipeline that finds its barrier not
+ *                  yet complete; 0 = the default (2 s), at most
+ *                  GL_WAIT_LIMIT_MAX_US.  A wait that runs out ORs
  *                  GL_DEV_TIMEOUT into the status word and the kernel stops
- *                  early with its outputs incomplete.  It exists to exercise
- *                  that failure path; the waits that drain a CTA's in-flight
- *                  copies and MMAs before it exits keep their 2 s bound.
+ *                  early with its outputs incomplete; the waits that drain a
+ *                  CTA's in-flight copies and MMAs before it exits keep their
+ *                  2 s bound.
+ *   flags          0, or GL_OPT_HOLD_LOADS: the load warp issues no copies,
+ *                  so no stage ever lands, every pipeline wait runs out after
+ *                  wait_limit_us, the call writes no output and sets
+ *                  GL_DEV_TIMEOUT.  It exists to test that failure path
+ *                  (status reported, context still usable) without a fault.
  * Values the header does not define give GL_ERR_INVALID.
  */
 #define GL_TILES_PAIR 0
 #define GL_TILES_SINGLE 1
 #define GL_WAIT_LIMIT_MAX_US 2000000u
+#define GL_OPT_HOLD_LOADS 1u
 typedef struct gl_gemm_opts {
   int tiles;
   uint32_t wait_limit_us;
+  uint32_t flags;
 } gl_gemm_opts;
 
 /*

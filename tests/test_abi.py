@@ -74,8 +74,9 @@ def test_gemm_options_are_checked():
     lib = gl.load()
     w = gl.GlGrouped(gl.GL_STACKED, 16, None)
     bad_tiles = ctypes.pointer(gl.GlGemmOpts(7, 0))
-    too_long = ctypes.pointer(gl.GlGemmOpts(gl.GL_TILES_PAIR, 2000001))
-    for o in (bad_tiles, too_long):
+    too_long = ctypes.pointer(gl.GlGemmOpts(gl.GL_TILES_PAIR, 2000001, 0))
+    bad_flags = ctypes.pointer(gl.GlGemmOpts(gl.GL_TILES_PAIR, 0, 6))
+    for o in (bad_tiles, too_long, bad_flags):
         assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 8, 8, 16, 8, o, None) == gl.GL_ERR_INVALID
         assert lib.gl_dgrad(16, w, 16, 16, 2, 8, 8, 8, 16, 8, o, None) == gl.GL_ERR_INVALID
         assert lib.gl_wgrad(16, 16, 16, 16, 2, 8, 8, 8, w, 1, o, None) == gl.GL_ERR_INVALID
@@ -83,7 +84,7 @@ def test_gemm_options_are_checked():
         assert lib.gl_dgrad_mxfp8(16, 16, w, w, 16, 16, 2, 8, 128, 128, 16, 8, o, None) == gl.GL_ERR_INVALID
         assert lib.gl_wgrad_mxfp8(16, 16, 16, 16, 16, 16, 2, 8, 128, 128, w, 1, o, None) == gl.GL_ERR_INVALID
     # no rows: valid options (and NULL) return before any launch
-    ok = ctypes.pointer(gl.GlGemmOpts(gl.GL_TILES_SINGLE, 1))
+    ok = ctypes.pointer(gl.GlGemmOpts(gl.GL_TILES_SINGLE, 1, gl.GL_OPT_HOLD_LOADS))
     for o in (None, ok):
         assert lib.gl_fwd(16, w, None, 16, 16, 2, 0, 8, 8, 16, 0, o, None) == gl.GL_OK
         assert lib.gl_dgrad(16, w, 16, 16, 2, 0, 8, 8, 16, 0, o, None) == gl.GL_OK

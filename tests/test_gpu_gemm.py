@@ -271,24 +271,27 @@ def test_full_size_sampled(name, pair):
 
 @pytest.mark.parametrize("pair_", [False, True], ids=["single", "pair"])
 def test_pipeline_wait_timeout_sets_status_and_recovers(pair_):
-    """With the per-call pipeline wait bound at 1 us the first tile's
-    accumulator (64 k-blocks of loads and MMAs) cannot be ready in time: the
-    epilogue's wait runs out, GL_DEV_TIMEOUT is ORed into the status word and
-    the kernel returns (every drain of in-flight copies and MMAs keeps its own
-    bound).  The same call with the default bound then matches the oracle."""
-    G, N, K, m = 3, 512, 4096, [300, 0, 212]
+    """A call whose load warp is held (GL_OPT_HOLD_LOADS: no stage ever
+    lands) with its pipeline waits bounded at 2 ms: every wait runs out,
+    GL_DEV_TIMEOUT is ORed into the status word, the kernel returns, and it
+    writes nothing (the output buffer keeps its sentinel, main_grad its
+    bytes).  The same calls with the default options then match the oracle:
+    the context is still usable."""
+    G, N, K, m = 3, 512, 1024, [300, 0, 212]
     M = sum(m)
     d = _inputs(G, N, K, m, seed=41)
     off, st = offsets_on_device(m, M)
     y = sentinel_like(M, N)
-    gl.gl_fwd(d["x"], d["w"], d["bias"], off, st, y, pair=pair_, wait_limit_us=1)
     mg = d["main_grad"].clone()
-    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True, pair=pair_, wait_limit_us=1)
+    hold = dict(pair=pair_, wait_limit_us=2000, opt_flags=gl.GL_OPT_HOLD_LOADS)
+    gl.gl_fwd(d["x"], d["w"], d["bias"], off, st, y, **hold)
+    gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True, **hold)
     torch.cuda.synchronize()
-    assert int(st.item()) & gl.GL_DEV_TIMEOUT
+    assert int(st.item()) == gl.GL_DEV_TIMEOUT
+    assert untouched(y)
+    assert torch.equal(mg, d["main_grad"])
     st.zero_()
     gl.gl_fwd(d["x"], d["w"], d["bias"], off, st, y, pair=pair_)
-    mg = d["main_grad"].clone()
     gl.gl_wgrad(d["x"], d["dy"], off, st, mg, accumulate=True, pair=pair_)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
@@ -300,4 +303,3 @@ def test_pipeline_wait_timeout_sets_status_and_recovers(pair_):
     for g in range(G):
         if m[g]:
             assert orc.rel_frobenius(got[g] - mg0[g], ref[g] - mg0[g]) <= TOL_BF16, g
-

@@ -173,6 +173,45 @@ def test_mxfp8_integer_mode_bit_exact(pair):
     assert np.array_equal(f64(mg), orc.wgrad(x64, dy64, m, f64(d["main_grad"]), True))
 
 
+@pytest.mark.parametrize("pair_", [False, True], ids=["single", "pair"])
+def test_mxfp8_wait_timeout_sets_status_and_recovers(pair_):
+    """GL_OPT_HOLD_LOADS with 2 ms pipeline waits on the MXFP8 GEMMs: the
+    status word gets GL_DEV_TIMEOUT and nothing is written; the same calls
+    with the default options then match the oracle."""
+    G, N, K, m = 3, 256, 512, [300, 0, 212]
+    M = sum(m)
+    d = {k: v.cuda() for k, v in synth.operands(G, M, N, K, seed=43, bias=True).items()}
+    off, st = offsets_on_device(m, M)
+    q = _quantize_all(d, m, G, N, K, off, st)
+    torch.cuda.synchronize()
+    args_f = (q["x"]["codes_r"], q["x"]["scales_r"], q["w"]["codes_r"].view(G, N, K), q["w"]["scales_r"],
+              d["bias"], off, st)
+    args_w = (q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st)
+    y = sentinel_like(M, N)
+    mg = d["main_grad"].clone()
+    hold = dict(pair=pair_, wait_limit_us=2000, opt_flags=gl.GL_OPT_HOLD_LOADS)
+    gl.gl_fwd_mxfp8(*args_f, y, **hold)
+    gl.gl_wgrad_mxfp8(*args_w, mg, accumulate=True, **hold)
+    torch.cuda.synchronize()
+    assert int(st.item()) == gl.GL_DEV_TIMEOUT
+    assert untouched(y)
+    assert torch.equal(mg, d["main_grad"])
+    st.zero_()
+    gl.gl_fwd_mxfp8(*args_f, y, pair=pair_)
+    gl.gl_wgrad_mxfp8(*args_w, mg, accumulate=True, pair=pair_)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = _oracle_all(d, m, G, N, K)
+    o = orc.offsets(m)
+    got_y, got_w, mg0 = f64(y), f64(mg), f64(d["main_grad"])
+    for g in range(G):
+        a, b = int(o[g]), int(o[g + 1])
+        if a == b:
+            continue
+        assert orc.rel_frobenius(got_y[a:b], ref["fwd"][a:b]) <= TOL_MX, ("fwd", g)
+        assert orc.rel_frobenius(got_w[g] - mg0[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad", g)
+
+
 FULL_MX = ["mxfp8_g8", "stacked_g128_uniform", "stacked_g128_ragged"]
 ROWS_PER_GROUP = 8   # random rows per group, besides the group's first and last row
 COLS = 64            # output columns sampled per group
