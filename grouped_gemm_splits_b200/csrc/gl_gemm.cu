@@ -49,9 +49,11 @@ struct Cfg {
   static constexpr int kTileM = 128 * CG;          // accumulator rows per tile (pair)
   static constexpr int kTileN = 256;               // accumulator columns
   static constexpr int kBRows = kTileN / CG;       // rows of the B operand held per CTA
-  // contraction elements per stage; only wgrad, whose operands are both
-  // MN-major, could take longer stages (a K-major box spans one 128-byte row)
-  static constexpr int kBK = BK;
+  // contraction elements per stage.  A K-major box spans one 128-byte row, so
+  // fwd / dgrad stages hold 64; wgrad on CTA pairs, whose operands are both
+  // MN-major, takes 128-row stages (three of them): half the barrier round
+  // trips and TMA boxes per flop, ~10% faster over the 8-group wgrad
+  static constexpr int kBK = (MODE == kWgrad && CG == 2) ? 128 : BK;
   static constexpr int kMNChunk = 128 * kBK;        // bytes of a 64-column MN-major chunk of a stage
   static constexpr int kABytes = 128 * kBK * 2;     // 16 KB
   static constexpr int kBBytes = kBRows * kBK * 2;  // 32 KB (CG 1) or 16 KB (CG 2)

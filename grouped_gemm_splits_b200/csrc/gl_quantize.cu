@@ -10,7 +10,7 @@
 //
 // Work unit: a 32-row block of one group (the columnwise block) x 256
 // columns (16 KB of bf16).  The kernel is persistent; one thread of each CTA
-// keeps a ring of kQStages tiles loaded ahead by TMA (mbarrier completion),
+// keeps a ring of tiles loaded ahead by TMA (mbarrier completion),
 // and the CTA's 256 threads read each element once from shared memory (a
 // thread: 4 rows x 8 columns).  Rowwise amax is a 4-lane shuffle reduction,
 // columnwise amax a shared-memory reduction over the block's 32 rows.  Each
@@ -39,24 +39,38 @@ constexpr int kQCols = 256;
 constexpr int kQRows = 32;
 constexpr int kQTileBytes = kQRows * kQCols * 2;  // one work unit of bf16
 static_assert(kQThreads == 256 && kQCols == 256, "one column per thread; 8 warps x 4 rows = 32 rows");
-constexpr int kQStages = 4;     // tiles staged in shared memory by TMA
-constexpr int kQCtasPerSm = 2;  // 2 x 4 x 16 KB of loads in flight per SM
+// Tiles staged in shared memory by TMA, and CTAs per SM: the plain cast fits
+// three CTAs (24 warps) in 80 registers a thread, which keeps more of the
+// per-tile dependency chains (amax -> scale -> convert) in flight; with the
+// bias-gradient sums it keeps two CTAs and four stages.
+template <bool kDbias>
+struct QCfg {
+  static constexpr int kStages = kDbias ? 4 : 3;
+  static constexpr int kCtasPerSm = kDbias ? 2 : 3;
+};
 
-// Scale exponent: the smallest e with amax <= 448 * 2^e, clamped to
-// [-127, 127].  448 = 1.75 * 2^8, so for amax = 1.m * 2^(E-127) the answer is
-// E - 135, plus one when 1.m > 1.75; a subnormal amax (E = 0) is below
-// 448 * 2^-127; amax = 0 gives 0.  Branch-free (selects only).
-__device__ __forceinline__ int mx_scale_exp(float amax) {
-  const uint32_t b = __float_as_uint(amax);
-  const int E = static_cast<int>(b >> 23);
-  const int e = max(E - 135 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0), -127);
-  return b == 0 ? 0 : e;
+// Per 16-bit half: the unsigned maximum.
+__device__ __forceinline__ uint32_t umax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
-// 2^-e as a float; e in [-127, 120] (the range finite bf16 amax values give)
-// is a normal number.
-__device__ __forceinline__ float pow2_neg(int e) {
-  return __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+// The two bf16 values of a word as fp32 (a bf16 is the high half of an fp32).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Block scale from the bf16 bits `a` of a block's amax (sign clear): the
+// smallest e with amax <= 448 * 2^e, clamped to [-127, 127]; e = 0 when
+// amax = 0.  448 = 1.75 * 2^8, so for amax = 1.m * 2^(E-127) the answer is
+// E - 135, plus one when 1.m > 1.75, i.e. when the 7 mantissa bits exceed
+// 0x60: adding 0x1F carries into the exponent field exactly then.  A
+// subnormal amax is below 448 * 2^-127.  Returns 2^-e as a float and the
+// biased byte e + 127.
+__device__ __forceinline__ float mx_scale_bf16(uint32_t a, uint32_t& byte) {
+  const uint32_t ec = max((a + 0x1Fu) >> 7, 8u);  // e + 135, at least 8
+  byte = a ? ec - 8u : 127u;
+  return __uint_as_float(a ? (262u - ec) << 23 : 0x3F800000u);
 }
 
 // (a, b) * (sa, sb) with one packed fp32 multiply (exact here: the scales
@@ -76,32 +90,37 @@ __device__ __forceinline__ uint32_t e4m3x2_scaled(float a, float b, float sa, fl
   return q;
 }
 
-// Eight values times their scales -> eight E4M3 codes (first value lowest).
-__device__ __forceinline__ uint2 e4m3x8(const float (&v)[8], const float (&sc)[8]) {
+// Eight bf16 values (four words, first value lowest) times one scale ->
+// eight E4M3 codes.
+__device__ __forceinline__ uint2 e4m3x8(const uint4& w, float sc) {
   uint2 q;
-  q.x = e4m3x2_scaled(v[0], v[1], sc[0], sc[1]) | (e4m3x2_scaled(v[2], v[3], sc[2], sc[3]) << 16);
-  q.y = e4m3x2_scaled(v[4], v[5], sc[4], sc[5]) | (e4m3x2_scaled(v[6], v[7], sc[6], sc[7]) << 16);
+  q.x = e4m3x2_scaled(bf16_lo(w.x), bf16_hi(w.x), sc, sc) | (e4m3x2_scaled(bf16_lo(w.y), bf16_hi(w.y), sc, sc) << 16);
+  q.y = e4m3x2_scaled(bf16_lo(w.z), bf16_hi(w.z), sc, sc) | (e4m3x2_scaled(bf16_lo(w.w), bf16_hi(w.w), sc, sc) << 16);
   return q;
 }
 
-// max |v| over eight values, as a balanced tree (short dependency chains).
-__device__ __forceinline__ float amax8(const float (&v)[8]) {
-  const float a = fmaxf(fabsf(v[0]), fabsf(v[1])), b = fmaxf(fabsf(v[2]), fabsf(v[3]));
-  const float c = fmaxf(fabsf(v[4]), fabsf(v[5])), d = fmaxf(fabsf(v[6]), fabsf(v[7]));
-  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+// Same, value j scaled by its column's scale (s0: columns 0-3, s1: 4-7).
+__device__ __forceinline__ uint2 e4m3x8(const uint4& w, const float4& s0, const float4& s1) {
+  uint2 q;
+  q.x = e4m3x2_scaled(bf16_lo(w.x), bf16_hi(w.x), s0.x, s0.y) |
+        (e4m3x2_scaled(bf16_lo(w.y), bf16_hi(w.y), s0.z, s0.w) << 16);
+  q.y = e4m3x2_scaled(bf16_lo(w.z), bf16_hi(w.z), s1.x, s1.y) |
+        (e4m3x2_scaled(bf16_lo(w.w), bf16_hi(w.w), s1.z, s1.w) << 16);
+  return q;
 }
 
 // kDbias: also write the per-block column sums (part: [part_blocks, cols]
 // fp32, block b of the launch in row b; part_prefix: the groups' first
 // blocks, int64[G+1], written by CTA 0).
 template <bool kDbias>
-__global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
+__global__ void __launch_bounds__(kQThreads, QCfg<kDbias>::kCtasPerSm)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_src, int64_t rows, int cols, int box_rows,
                     int tile_bytes, const int64_t* __restrict__ row_offsets, int G, int32_t* status,
                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r,
                     uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, int64_t scales_c_bytes,
                     int mma_layout, float* __restrict__ part, int64_t part_blocks,
                     int64_t* __restrict__ part_prefix) {
+  constexpr int kQStages = QCfg<kDbias>::kStages;
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* qsmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_buf = qsmem;                                                  // kQStages x 16 KB
@@ -109,7 +128,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kQStages);
   int64_t* bprefix = reinterpret_cast<int64_t*>(qsmem + kQStages * kQTileBytes + 64);  // G+1 (ragged)
   int64_t* qprefix = bprefix + G + 1;                                                  // G+1 (ragged)
-  __shared__ __align__(16) float cmax[kQThreads / 32][kQCols];  // per-warp column maxima
+  __shared__ __align__(16) uint32_t cmax[kQThreads / 32][kQCols / 2];  // per-warp column maxima, bf16 pairs
   __shared__ __align__(16) float csf[kQCols];                     // 2^-e of each column
   __shared__ __align__(16) float csum[kDbias ? kQThreads / 32 : 1][kQCols];  // per-warp column sums
   if (status != nullptr && *reinterpret_cast<volatile int32_t*>(status) != 0) return;
@@ -242,6 +261,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     // end-of-tile barrier (every thread reaches it)
     if (!mbar_wait(&full[s], static_cast<uint32_t>(consumed / kQStages) & 1u, abort_flag)) *abort_flag = 1;
     const bool work = *abort_flag == 0;
+    // this thread's 4 rows x 8 columns, one 16-byte piece per row (rows past
+    // the block's valid rows read as zero)
     uint4 raw[4];
     {
       const uint8_t* tile = stage_buf + s * kQTileBytes + c8 * 16;
@@ -254,33 +275,40 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     }
     const int col = cc * kQCols + c8 * 8;
     const bool col_ok = work && col < cols;
-    float v[4][8];  // a bf16 is the high half of an fp32
+    // |v| as pairs of bf16 bit patterns: for non-negative values the unsigned
+    // order of the bits is the order of the values, so every block maximum
+    // is an integer maximum over 16-bit halves
+    uint32_t mag[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        v[i][2 * k] = __uint_as_float(w[k] << 16);
-        v[i][2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-      }
+      mag[i][0] = raw[i].x & 0x7FFF7FFFu;
+      mag[i][1] = raw[i].y & 0x7FFF7FFFu;
+      mag[i][2] = raw[i].z & 0x7FFF7FFFu;
+      mag[i][3] = raw[i].w & 0x7FFF7FFFu;
     }
     const int64_t tile_off = r0 * cols + col;  // element offset of this thread's first value
 
     if (codes_r != nullptr) {
+      // row maxima over this thread's 8 columns, two rows per word, then over
+      // the 4 lanes that share each 32-column block
+      uint32_t m[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m[i] = umax2(umax2(mag[i][0], mag[i][1]), umax2(mag[i][2], mag[i][3]));
+      uint32_t p01 = umax2(__byte_perm(m[0], m[1], 0x5410), __byte_perm(m[0], m[1], 0x7632));
+      uint32_t p23 = umax2(__byte_perm(m[2], m[3], 0x5410), __byte_perm(m[2], m[3], 0x7632));
+      p01 = umax2(p01, __shfl_xor_sync(0xffffffffu, p01, 1));
+      p23 = umax2(p23, __shfl_xor_sync(0xffffffffu, p23, 1));
+      p01 = umax2(p01, __shfl_xor_sync(0xffffffffu, p01, 2));
+      p23 = umax2(p23, __shfl_xor_sync(0xffffffffu, p23, 2));
+      const uint32_t am[4] = {p01 & 0xFFFFu, p01 >> 16, p23 & 0xFFFFu, p23 >> 16};
       uint8_t* dst = codes_r + tile_off + static_cast<int64_t>(rbase) * cols;
       uint32_t ebytes = 0;  // biased scale exponents of this thread's 4 rows, row i in byte i
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        float a = amax8(v[i]);
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));  // the 4 lanes of a 32-column block
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-        const int e = mx_scale_exp(a);
-        ebytes |= static_cast<uint32_t>(e + 127) << (8 * i);
-        const float sc = pow2_neg(e);
-        if (col_ok && rbase + i < vrows) {
-          const float scv[8] = {sc, sc, sc, sc, sc, sc, sc, sc};
-          *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(v[i], scv);
-        }
+        uint32_t byte;
+        const float sc = mx_scale_bf16(am[i], byte);
+        ebytes |= byte << (8 * i);
+        if (col_ok && rbase + i < vrows) *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(raw[i], sc);
       }
       // the warp's 4 rows x 8 blocks of 32 columns are 32 scales: lane L
       // writes the one of row L/8, block L%8 (taken from that block's first
@@ -307,7 +335,11 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     if (kDbias) {
       float cs[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) cs[k] = ((v[0][k] + v[1][k]) + v[2][k]) + v[3][k];
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t w0 = (&raw[0].x)[k], w1 = (&raw[1].x)[k], w2 = (&raw[2].x)[k], w3 = (&raw[3].x)[k];
+        cs[2 * k] = ((bf16_lo(w0) + bf16_lo(w1)) + bf16_lo(w2)) + bf16_lo(w3);
+        cs[2 * k + 1] = ((bf16_hi(w0) + bf16_hi(w1)) + bf16_hi(w2)) + bf16_hi(w3);
+      }
       float4* cp = reinterpret_cast<float4*>(&csum[warp][c8 * 8]);
       cp[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
       cp[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
@@ -322,47 +354,48 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     };
 
     if (codes_c != nullptr) {
-      float4* cm = reinterpret_cast<float4*>(&cmax[warp][c8 * 8]);
-      float c[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        c[k] = fmaxf(fmaxf(fabsf(v[0][k]), fabsf(v[1][k])), fmaxf(fabsf(v[2][k]), fabsf(v[3][k])));
-      cm[0] = make_float4(c[0], c[1], c[2], c[3]);
-      cm[1] = make_float4(c[4], c[5], c[6], c[7]);
+      // column maxima over this thread's 4 rows (two columns per word), then
+      // over the 8 warps through shared memory: thread t < 128 finishes
+      // columns 2t and 2t + 1 of the tile
+      uint4 cm;
+      cm.x = umax2(umax2(mag[0][0], mag[1][0]), umax2(mag[2][0], mag[3][0]));
+      cm.y = umax2(umax2(mag[0][1], mag[1][1]), umax2(mag[2][1], mag[3][1]));
+      cm.z = umax2(umax2(mag[0][2], mag[1][2]), umax2(mag[2][2], mag[3][2]));
+      cm.w = umax2(umax2(mag[0][3], mag[1][3]), umax2(mag[2][3], mag[3][3]));
+      reinterpret_cast<uint4*>(cmax[warp])[c8] = cm;
       __syncthreads();
-      {
-        float p[kQThreads / 32];
+      if (tid < kQCols / 2) {
+        uint32_t a = cmax[0][tid];
 #pragma unroll
-        for (int w = 0; w < kQThreads / 32; ++w) p[w] = cmax[w][tid];
-        const float a = fmaxf(fmaxf(fmaxf(p[0], p[1]), fmaxf(p[2], p[3])), fmaxf(fmaxf(p[4], p[5]), fmaxf(p[6], p[7])));
-        const int e = mx_scale_exp(a);
-        csf[tid] = pow2_neg(e);
-        const int ccol = cc * kQCols + tid;
-        if (work && ccol < cols && vrows > 0) {
-          int64_t at;
-          if (mma_layout) {
-            // atom (k-group of the group's blocks 4t..4t+3, 128 columns)
-            const int64_t kq = (ragged ? qprefix[g] : static_cast<int64_t>(g) * qpg) + (j >> 2);
-            at = (kq * mma_cb + (ccol >> 7)) * 512 + (((ccol & 31) << 4) | (((ccol >> 5) & 3) << 2) | (j & 3));
-          } else {
-            at = ((ragged ? bprefix[g] : static_cast<int64_t>(g) * bpg) + j) * cols + ccol;
+        for (int w = 1; w < kQThreads / 32; ++w) a = umax2(a, cmax[w][tid]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t byte;
+          csf[2 * tid + h] = mx_scale_bf16(h ? (a >> 16) : (a & 0xFFFFu), byte);
+          const int ccol = cc * kQCols + 2 * tid + h;
+          if (work && ccol < cols && vrows > 0) {
+            int64_t at;
+            if (mma_layout) {
+              // atom (k-group of the group's blocks 4t..4t+3, 128 columns)
+              const int64_t kq = (ragged ? qprefix[g] : static_cast<int64_t>(g) * qpg) + (j >> 2);
+              at = (kq * mma_cb + (ccol >> 7)) * 512 + (((ccol & 31) << 4) | (((ccol >> 5) & 3) << 2) | (j & 3));
+            } else {
+              at = ((ragged ? bprefix[g] : static_cast<int64_t>(g) * bpg) + j) * cols + ccol;
+            }
+            // offsets that overlap (only possible without a status word) must
+            // not push a write past the documented allocation
+            if (at < scales_c_bytes) scales_c[at] = static_cast<uint8_t>(byte);
           }
-          // offsets that overlap (only possible without a status word) must
-          // not push a write past the documented allocation
-          if (at < scales_c_bytes) scales_c[at] = static_cast<uint8_t>(e + 127);
         }
       }
       if (kDbias) store_partial();  // csum complete since the barrier above
       __syncthreads();
       const float4 s0 = reinterpret_cast<const float4*>(csf)[c8 * 2];
       const float4 s1 = reinterpret_cast<const float4*>(csf)[c8 * 2 + 1];
-      const float scc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
       uint8_t* dst = codes_c + tile_off + static_cast<int64_t>(rbase) * cols;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        if (col_ok && rbase + i < vrows) {
-          *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(v[i], scc);
-        }
+        if (col_ok && rbase + i < vrows) *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(raw[i], s0, s1);
       }
     }
     if (kDbias && codes_c == nullptr) {
@@ -404,20 +437,22 @@ gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t
   const uint32_t box[2] = {box_cols, box_rows};
   if (!encode_tmap(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, src, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
     return GL_ERR_UNSUPPORTED;
-  const int smem = 1024 + kQStages * kQTileBytes + 64 +
-                   (row_offsets != nullptr ? 2 * (G + 1) * static_cast<int>(sizeof(int64_t)) : 0);
-  const int grid = num_sms() * kQCtasPerSm;
+  const int prefix_bytes = row_offsets != nullptr ? 2 * (G + 1) * static_cast<int>(sizeof(int64_t)) : 0;
   const int tile_bytes = static_cast<int>(box_cols * box_rows * 2);
   const int64_t sc_bytes = static_cast<int64_t>(gl_mxfp8_scale_bytes(rows, cols, G, 1, scale_layout));
   const int mma = scale_layout == GL_SCALES_MMA ? 1 : 0;
   if (part != nullptr) {
+    using Q = QCfg<true>;
+    const int smem = 1024 + Q::kStages * kQTileBytes + 64 + prefix_bytes;
     if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel<true>), smem) != cudaSuccess) return GL_ERR_CUDA;
-    quantize_kernel<true><<<grid, kQThreads, smem, stream>>>(
+    quantize_kernel<true><<<num_sms() * Q::kCtasPerSm, kQThreads, smem, stream>>>(
         tm, rows, cols, static_cast<int>(box_rows), tile_bytes, row_offsets, G, status, codes_r, scales_r, codes_c,
         scales_c, sc_bytes, mma, part, part_blocks, part_prefix);
   } else {
+    using Q = QCfg<false>;
+    const int smem = 1024 + Q::kStages * kQTileBytes + 64 + prefix_bytes;
     if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel<false>), smem) != cudaSuccess) return GL_ERR_CUDA;
-    quantize_kernel<false><<<grid, kQThreads, smem, stream>>>(
+    quantize_kernel<false><<<num_sms() * Q::kCtasPerSm, kQThreads, smem, stream>>>(
         tm, rows, cols, static_cast<int>(box_rows), tile_bytes, row_offsets, G, status, codes_r, scales_r, codes_c,
         scales_c, sc_bytes, mma, nullptr, 0, nullptr);
   }
