@@ -44,6 +44,10 @@ def test_host_side_validation_without_gpu():
     assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 12, 8, 16, 8, None, None) == gl.GL_ERR_UNSUPPORTED
     # caller buffer with fewer rows than the input
     assert lib.gl_fwd(16, w, None, 16, 16, 2, 8, 8, 8, 16, 7, None, None) == gl.GL_ERR_INVALID
+    # more groups than the kernels take
+    assert lib.gl_fwd(16, w, None, 16, 16, 4097, 8, 8, 8, 16, 8, None, None) == gl.GL_ERR_INVALID
+    assert lib.gl_offsets(16, 4097, 8, 8, 16, 16, None) == gl.GL_ERR_INVALID
+    assert lib.gl_fwd_mxfp8(16, 16, w, w, None, 16, 16, 2049, 8, 128, 128, 16, 8, None, None) == gl.GL_ERR_INVALID
     # null pointers
     assert lib.gl_fwd(None, w, None, 16, 16, 2, 8, 8, 8, 16, 8, None, None) == gl.GL_ERR_INVALID
     assert lib.gl_dgrad(16, w, 16, None, 2, 8, 8, 8, 16, 8, None, None) == gl.GL_ERR_INVALID

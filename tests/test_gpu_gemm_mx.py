@@ -212,6 +212,39 @@ def test_mxfp8_wait_timeout_sets_status_and_recovers(pair_):
         assert orc.rel_frobenius(got_w[g] - mg0[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad", g)
 
 
+def test_mxfp8_max_groups_stacked(pair):
+    """GL_MAX_GROUPS_MXFP8 (2048) groups in one stacked call, most of them
+    empty or short: the scale k-groups of the columnwise operands restart at
+    every group; each non-empty group checked on its own."""
+    rng = np.random.default_rng(2048)
+    G, N, K = 2048, 128, 128
+    m = [int(v) for v in synth.random_splits(rng, G, 12000, p_empty=0.5)]
+    M = sum(m)
+    d = {k: v.cuda() for k, v in synth.operands(G, M, N, K, seed=2048, bias=True).items()}
+    off, st = offsets_on_device(m, M)
+    q = _quantize_all(d, m, G, N, K, off, st)
+    y = gl.gl_fwd_mxfp8(q["x"]["codes_r"], q["x"]["scales_r"], q["w"]["codes_r"].view(G, N, K), q["w"]["scales_r"],
+                        d["bias"], off, st, pair=pair)
+    dx = gl.gl_dgrad_mxfp8(q["dy"]["codes_r"], q["dy"]["scales_r"], q["w"]["codes_c"].view(G, N, K),
+                           q["w"]["scales_c"], off, st, pair=pair)
+    mg = torch.full((G, N, K), float("nan"), device="cuda")
+    gl.gl_wgrad_mxfp8(q["x"]["codes_c"], q["x"]["scales_c"], q["dy"]["codes_c"], q["dy"]["scales_c"], off, st, mg,
+                      accumulate=False, pair=pair)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = _oracle_all(d, m, G, N, K)
+    o = orc.offsets(m)
+    got_y, got_dx, got_w = f64(y), f64(dx), f64(mg)
+    for g in range(G):
+        a, b = int(o[g]), int(o[g + 1])
+        if a == b:
+            assert np.all(got_w[g] == 0.0), g
+            continue
+        assert orc.rel_frobenius(got_y[a:b], ref["fwd"][a:b]) <= TOL_MX, ("fwd", g)
+        assert orc.rel_frobenius(got_dx[a:b], ref["dgrad"][a:b]) <= TOL_MX, ("dgrad", g)
+        assert orc.rel_frobenius(got_w[g], ref["wgrad_over"][g]) <= TOL_MX, ("wgrad", g)
+
+
 FULL_MX = ["mxfp8_g8", "stacked_g128_uniform", "stacked_g128_ragged"]
 ROWS_PER_GROUP = 8   # random rows per group, besides the group's first and last row
 COLS = 64            # output columns sampled per group
