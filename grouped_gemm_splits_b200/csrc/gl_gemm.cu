@@ -41,7 +41,7 @@ namespace {
 
 constexpr int BK = 64;  // contraction elements of a K-major stage (one 128-byte swizzle row)
 constexpr int kPG = 64;  // per-group tensor maps carried by one launch
-constexpr int kSmemBudget = 212992;  // 6 stages of 32 KB + (wgrad) 16 KB of epilogue transposes
+constexpr int kSmemBudget = 212992;  // stage ring (pairs: 3 x 64 KB; single CTAs: 4 x 48 KB) + (wgrad) 16 KB of transposes
 constexpr int kBand = 8;  // tile rows per rasterisation band
 
 template <int MODE, int CG>
@@ -49,14 +49,15 @@ struct Cfg {
   static constexpr int kTileM = 128 * CG;          // accumulator rows per tile (pair)
   static constexpr int kTileN = 256;               // accumulator columns
   static constexpr int kBRows = kTileN / CG;       // rows of the B operand held per CTA
-  // contraction elements per stage.  A K-major box spans one 128-byte row, so
-  // fwd / dgrad stages hold 64; wgrad on CTA pairs, whose operands are both
-  // MN-major, takes 128-row stages (three of them): half the barrier round
-  // trips and TMA boxes per flop, ~10% faster over the 8-group wgrad
-  static constexpr int kBK = (MODE == kWgrad && CG == 2) ? 128 : BK;
+  // contraction elements per stage.  A K-major box spans one 128-byte row (64
+  // elements); on CTA pairs a stage holds 128 (two boxes per K-major operand,
+  // three stages of 64 KB): half the barrier round trips per flop, ~10%
+  // faster for wgrad (both operands MN-major) and ~2.5% for fwd / dgrad.
+  // Single CTAs keep 64, which leaves room for four 48 KB stages.
+  static constexpr int kBK = (CG == 2) ? 128 : BK;
   static constexpr int kMNChunk = 128 * kBK;        // bytes of a 64-column MN-major chunk of a stage
-  static constexpr int kABytes = 128 * kBK * 2;     // 16 KB
-  static constexpr int kBBytes = kBRows * kBK * 2;  // 32 KB (CG 1) or 16 KB (CG 2)
+  static constexpr int kABytes = 128 * kBK * 2;     // 32 KB (CG 2) or 16 KB (CG 1)
+  static constexpr int kBBytes = kBRows * kBK * 2;  // 32 KB
   static constexpr int kStageBytes = kABytes + kBBytes;
   // epilogue warps, one per TMEM lane quarter (eight for wgrad measured no
   // faster and cost a pipeline stage of staging space)
@@ -78,8 +79,8 @@ struct Cfg {
 };
 
 struct GemmParams {
-  CUtensorMap tmA;    // FWD x{K,M} box{64,128}; DGRAD dy{N,M} box{64,128}; WGRAD dy{N,M} box{64,64}
-  CUtensorMap tmB;    // stacked W{K,N,G}: FWD box{64,BRows,1}, DGRAD box{64,64,1}; WGRAD x{K,M} box{64,64}
+  CUtensorMap tmA;    // FWD x{K,M} box{64,128}; DGRAD dy{N,M} box{64,128}; WGRAD dy{N,M} box{64,kBK}
+  CUtensorMap tmB;    // stacked W{K,N,G}: FWD box{64,BRows,1}, DGRAD box{64,kBK,1}; WGRAD x{K,M} box{64,kBK}
   const int64_t* offsets;  // G+1 entries
   int32_t* status;
   int64_t M;
@@ -169,7 +170,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const Gemm
   } else {
     tl.r0 = o0 + static_cast<int64_t>(tl.mt) * C::kTileM;
     tl.r1 = o0 + m;
-    tl.num_kb = ceil_div_i(MODE == kFwd ? p.K : p.N, BK);
+    tl.num_kb = ceil_div_i(MODE == kFwd ? p.K : p.N, C::kBK);
   }
   return tl;
 }
@@ -319,16 +320,21 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
           if (MODE == kFwd) {
             const int n0 = tl.nt * C::kTileN + hb;
-            tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0 + hr));
-            if (PG) tma_load_2d(sb, pg.map(tl.g), &full[stage], kb * BK, n0);
-            else    tma_load_3d(sb, &p.tmB, &full[stage], kb * BK, n0, tl.g);
+#pragma unroll
+            for (int c = 0; c < C::kBK / 64; ++c) {
+              tma_load_2d(sa + c * 16384, &p.tmA, &full[stage], kb * C::kBK + c * 64, static_cast<int32_t>(tl.r0 + hr));
+              if (PG) tma_load_2d(sb + c * C::kBRows * 128, pg.map(tl.g), &full[stage], kb * C::kBK + c * 64, n0);
+              else    tma_load_3d(sb + c * C::kBRows * 128, &p.tmB, &full[stage], kb * C::kBK + c * 64, n0, tl.g);
+            }
           } else if (MODE == kDgrad) {
             const int n0 = tl.nt * C::kTileN + hb;
-            tma_load_2d(sa, &p.tmA, &full[stage], kb * BK, static_cast<int32_t>(tl.r0 + hr));
+#pragma unroll
+            for (int c = 0; c < C::kBK / 64; ++c)
+              tma_load_2d(sa + c * 16384, &p.tmA, &full[stage], kb * C::kBK + c * 64, static_cast<int32_t>(tl.r0 + hr));
 #pragma unroll
             for (int c = 0; c < C::kBRows / 64; ++c) {
-              if (PG) tma_load_2d(sb + c * C::kMNChunk, pg.map(tl.g), &full[stage], n0 + c * 64, kb * BK);
-              else    tma_load_3d(sb + c * C::kMNChunk, &p.tmB, &full[stage], n0 + c * 64, kb * BK, tl.g);
+              if (PG) tma_load_2d(sb + c * C::kMNChunk, pg.map(tl.g), &full[stage], n0 + c * 64, kb * C::kBK);
+              else    tma_load_3d(sb + c * C::kMNChunk, &p.tmB, &full[stage], n0 + c * 64, kb * C::kBK, tl.g);
             }
           } else {
             // operand strips are read again by the neighbouring tiles of the
@@ -407,9 +413,9 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
             const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
             for (int ks = 0; ks < ksteps; ++ks) {
               const uint64_t ad = C::kAMN ? smem_desc_sw128(a0 + ks * 2048, C::kMNChunk, 1024)
-                                          : smem_desc_sw128(a0 + ks * 32, 16, 1024);
+                                          : smem_desc_sw128(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
               const uint64_t bd = C::kBMN ? smem_desc_sw128(b0 + ks * 2048, C::kMNChunk, 1024)
-                                          : smem_desc_sw128(b0 + ks * 32, 16, 1024);
+                                          : smem_desc_sw128(b0 + (ks >> 2) * (C::kBRows * 128) + (ks & 3) * 32, 16, 1024);
               const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
               if (CG == 2) mma_bf16_ss_pair(d_tmem, ad, bd, C::kIdesc, acc);
               else         mma_bf16_ss(d_tmem, ad, bd, C::kIdesc, acc);
@@ -729,7 +735,7 @@ gl_status launch_mode(const GemmCall& c) {
   const bool bias_stacked = prm.has_bias && c.bias->mode == GL_STACKED;
   if (stacked && (!prm.has_bias || bias_stacked)) {
     if (MODE == kFwd) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, BK, Cf::kBRows, BF, 2);
-    if (MODE == kDgrad) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, 64, BK, BF, 2);
+    if (MODE == kDgrad) ok &= make_3d(&prm.tmB, c.w.base, c.K, c.N, c.G, 64, Cf::kBK, BF, 2);
     if (MODE == kWgrad) prm.mg = static_cast<float*>(const_cast<void*>(c.out_grouped.base));
     if (!ok) return GL_ERR_UNSUPPORTED;
     prm.offsets = c.offsets;
@@ -751,7 +757,7 @@ gl_status launch_mode(const GemmCall& c) {
                              ? static_cast<const uint8_t*>(c.w.base) + static_cast<size_t>(g) * c.N * c.K * 2
                              : c.w.ptrs[g];
         if (MODE == kFwd) ok &= make_2d(&pga->tm[i], wp, c.K, c.N, BK, Cf::kBRows, BF, 2);
-        else              ok &= make_2d(&pga->tm[i], wp, c.K, c.N, 64, BK, BF, 2);
+        else              ok &= make_2d(&pga->tm[i], wp, c.K, c.N, 64, Cf::kBK, BF, 2);
         if (prm.has_bias)
           pga->bias[i] = reinterpret_cast<const __nv_bfloat16*>(
               c.bias->mode == GL_STACKED
