@@ -410,15 +410,26 @@ __global__ void __launch_bounds__(Cfg<MODE, CG>::kThreads, 1)
           }
           __syncwarp();
           if (lane == 0) {
-            const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
-            for (int ks = 0; ks < ksteps; ++ks) {
-              const uint64_t ad = C::kAMN ? smem_desc_sw128(a0 + ks * 2048, C::kMNChunk, 1024)
-                                          : smem_desc_sw128(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-              const uint64_t bd = C::kBMN ? smem_desc_sw128(b0 + ks * 2048, C::kMNChunk, 1024)
-                                          : smem_desc_sw128(b0 + (ks >> 2) * (C::kBRows * 128) + (ks & 3) * 32, 16, 1024);
+            // The single issuing thread is on the critical path: descriptors
+            // are formed once per stage and advanced by constants (16-byte
+            // units: 16 MN-major rows of 128 bytes, or 16 K-major elements
+            // within a 64-element box, then the next box).
+            const uint64_t ad0 = C::kAMN ? smem_desc_sw128(smem_u32(sa), C::kMNChunk, 1024)
+                                         : smem_desc_sw128(smem_u32(sa), 16, 1024);
+            const uint64_t bd0 = C::kBMN ? smem_desc_sw128(smem_u32(sb), C::kMNChunk, 1024)
+                                         : smem_desc_sw128(smem_u32(sb), 16, 1024);
+            auto issue = [&](int ks) {
+              const uint32_t ao = C::kAMN ? ks * 128 : (ks >> 2) * 1024 + (ks & 3) * 2;
+              const uint32_t bo = C::kBMN ? ks * 128 : (ks >> 2) * (C::kBRows * 8) + (ks & 3) * 2;
               const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-              if (CG == 2) mma_bf16_ss_pair(d_tmem, ad, bd, C::kIdesc, acc);
-              else         mma_bf16_ss(d_tmem, ad, bd, C::kIdesc, acc);
+              if (CG == 2) mma_bf16_ss_pair(d_tmem, desc_add(ad0, ao), desc_add(bd0, bo), C::kIdesc, acc);
+              else         mma_bf16_ss(d_tmem, desc_add(ad0, ao), desc_add(bd0, bo), C::kIdesc, acc);
+            };
+            if (ksteps == C::kBK / 16) {
+#pragma unroll
+              for (int ks = 0; ks < C::kBK / 16; ++ks) issue(ks);
+            } else {
+              for (int ks = 0; ks < ksteps; ++ks) issue(ks);
             }
             // free the stage (in both CTAs) once these MMAs have read it
             if (CG == 2) tc_commit_pair_mc(&empty[stage], 0x3);

@@ -237,6 +237,15 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// A descriptor advanced by `units` 16-byte units.  Its start-address field
+// (bits 0-13: shared-memory address / 16) never carries out inside shared
+// memory, so only the low word changes.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t units) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(static_cast<uint32_t>(d) + units), "r"(static_cast<uint32_t>(d >> 32)));
+  return r;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 // a_mn / b_mn: 1 when the operand is stored MN-major in shared memory.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
