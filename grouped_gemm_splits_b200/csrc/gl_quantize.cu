@@ -8,21 +8,23 @@
 // ``group_quantize_mxfp8`` ("Improve device-init grouped linear module",
 // PR #3224).
 //
-// Work unit: a 32-row block of one group (the columnwise block) x 256
-// columns (16 KB of bf16).  The kernel is persistent; one thread of each CTA
-// keeps a ring of tiles loaded ahead by TMA (mbarrier completion),
-// and the CTA's 256 threads read each element once from shared memory (a
-// thread: 4 rows x 8 columns).  Rowwise amax is a 4-lane shuffle reduction,
-// columnwise amax a shared-memory reduction over the block's 32 rows.  Each
-// CTA first builds the per-group block prefixes in shared memory.
-// Memory-bound: 2 bytes read and up to 2 bytes (+1/16 for scales) written per
-// element.
+// Work unit (tile): a 32-row block of one group (the columnwise block) x 512
+// columns (256 when the rows are narrower), staged in shared memory by TMA.
+// The kernel is persistent; a producer warp keeps a ring of tiles loaded
+// ahead (full / empty mbarriers) and eight consumer warps share no data: each
+// owns whole 32-column blocks of the tile (a lane: 4 rows x 8 columns of a
+// block), so both block maxima -- along a row and down a column -- are warp
+// shuffles and no block-wide barrier is taken per tile.  Each CTA first
+// builds the per-group block prefixes in shared memory.  Memory-bound in
+// principle: 2 bytes read and up to 2 bytes (+1/16 for scales) written per
+// element; in practice about a fifth below the copy bandwidth, bound by the
+// per-element integer and conversion work.
 //
 // With a bias gradient (the cast of dy; fuser_backward sums each split of
 // grad_output over its rows next to quantizing it), the same pass also adds
-// every work unit's 32 rows per column in fp32 -- a thread its 4 rows, then
-// the 8 warps in order through shared memory -- and stores one fp32 partial
-// per (32-row block, column) in a caller workspace; dbias_partials_kernel
+// every block's 32 rows per column in fp32 -- a lane its 4 rows, then the 8
+// row groups of the warp by a butterfly -- and stores one fp32 partial per
+// (32-row block, column) in a caller workspace; dbias_partials_kernel
 // (gl_dbias.cu) adds each group's partials in block order.  The sums are
 // deterministic: no atomics, a fixed order at every level.
 #include <cuda_bf16.h>
@@ -37,16 +39,15 @@ namespace {
 constexpr int kQThreads = 256;
 constexpr int kQCols = 256;
 constexpr int kQRows = 32;
-constexpr int kQTileBytes = kQRows * kQCols * 2;  // one work unit of bf16
-static_assert(kQThreads == 256 && kQCols == 256, "one column per thread; 8 warps x 4 rows = 32 rows");
-// Tiles staged in shared memory by TMA, and CTAs per SM: the plain cast fits
-// three CTAs (24 warps) in 80 registers a thread, which keeps more of the
-// per-tile dependency chains (amax -> scale -> convert) in flight; with the
-// bias-gradient sums it keeps two CTAs and four stages.
-template <bool kDbias>
+static_assert(kQThreads == 256 && kQCols == 256, "eight consumer warps, one 32-column block each per box");
+// Tiles staged in shared memory by TMA, and CTAs per SM (each CTA: eight
+// consumer warps and a producer warp).
+constexpr int kQBoxBytes = kQRows * kQCols * 2;  // one TMA box: 32 rows x 256 columns
+template <bool kDbias, int kCB>
 struct QCfg {
-  static constexpr int kStages = kDbias ? 4 : 3;
-  static constexpr int kCtasPerSm = kDbias ? 2 : 3;
+  static constexpr int kTileBytes = kCB * kQBoxBytes;
+  static constexpr int kStages = kCB == 1 ? 4 : 3;
+  static constexpr int kCtasPerSm = kCB == 1 ? 3 : 2;
 };
 
 // Per 16-bit half: the unsigned maximum.
@@ -109,32 +110,44 @@ __device__ __forceinline__ uint2 e4m3x8(const uint4& w, const float4& s0, const 
   return q;
 }
 
+// Work unit (tile): a 32-row block of one group x kCB * 256 columns, staged
+// in shared memory by TMA (kCB boxes of 32 x 256).  Warp 8 is the producer:
+// one thread keeps a ring of kStages tiles in flight (full / empty mbarriers).
+// Warps 0-7 are consumers and share no data: warp w owns the 32-column
+// blocks w, w + 8, .. of the tile, so that both block maxima of its elements
+// -- along a row (32 columns) and down a column (32 rows) -- are reduced
+// within the warp by shuffles.  A lane holds rows 4 * (lane / 4) .. + 3 and
+// 8 columns (8 * (lane % 4) ..) of each of its blocks.
+//
 // kDbias: also write the per-block column sums (part: [part_blocks, cols]
 // fp32, block b of the launch in row b; part_prefix: the groups' first
 // blocks, int64[G+1], written by CTA 0).
-template <bool kDbias>
-__global__ void __launch_bounds__(kQThreads, QCfg<kDbias>::kCtasPerSm)
+template <bool kDbias, int kCB>
+__global__ void __launch_bounds__(kQThreads + 32, QCfg<kDbias, kCB>::kCtasPerSm)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_src, int64_t rows, int cols, int box_rows,
-                    int tile_bytes, const int64_t* __restrict__ row_offsets, int G, int32_t* status,
+                    int box_bytes, const int64_t* __restrict__ row_offsets, int G, int32_t* status,
                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r,
                     uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, int64_t scales_c_bytes,
                     int mma_layout, float* __restrict__ part, int64_t part_blocks,
                     int64_t* __restrict__ part_prefix) {
-  constexpr int kQStages = QCfg<kDbias>::kStages;
+  using Q = QCfg<kDbias, kCB>;
+  constexpr int kStages = Q::kStages;
+  constexpr int kTileCols = kCB * kQCols;
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* qsmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stage_buf = qsmem;                                                  // kQStages x 16 KB
-  uint64_t* full = reinterpret_cast<uint64_t*>(qsmem + kQStages * kQTileBytes);  // one barrier per stage
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kQStages);
-  int64_t* bprefix = reinterpret_cast<int64_t*>(qsmem + kQStages * kQTileBytes + 64);  // G+1 (ragged)
-  int64_t* qprefix = bprefix + G + 1;                                                  // G+1 (ragged)
-  __shared__ __align__(16) uint32_t cmax[kQThreads / 32][kQCols / 2];  // per-warp column maxima, bf16 pairs
-  __shared__ __align__(16) float csf[kQCols];                     // 2^-e of each column
-  __shared__ __align__(16) float csum[kDbias ? kQThreads / 32 : 1][kQCols];  // per-warp column sums
+  uint8_t* stage_buf = qsmem;                                                      // kStages x kCB boxes
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsmem + kStages * Q::kTileBytes);  // tile landed
+  uint64_t* empty = full + kStages;                                               // tile consumed (8 warps)
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  int64_t* bprefix = reinterpret_cast<int64_t*>(qsmem + kStages * Q::kTileBytes + 128);  // G+1 (ragged)
+  int64_t* qprefix = bprefix + G + 1;                                                    // G+1 (ragged)
   if (status != nullptr && *reinterpret_cast<volatile int32_t*>(status) != 0) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
-    for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kQThreads / 32);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -168,19 +181,16 @@ __global__ void __launch_bounds__(kQThreads, QCfg<kDbias>::kCtasPerSm)
   }
   __syncthreads();
   if (kDbias && blockIdx.x == 0 && row_offsets != nullptr)
-    for (int i = tid; i <= G; i += kQThreads) part_prefix[i] = bprefix[i];
+    for (int i = tid; i <= G; i += blockDim.x) part_prefix[i] = bprefix[i];
   const int64_t nblocks = (row_offsets != nullptr) ? bprefix[G] : bpg * G;
-  const int ncc = (cols + kQCols - 1) / kQCols;
+  const int ncc = (cols + kTileCols - 1) / kTileCols;
   const int64_t ntiles = nblocks * ncc;
-  const int c8 = lane;         // 8-column chunk within the 256-column tile
-  const int rbase = warp * 4;  // this thread's 4 rows within the 32-row block
-  const int pitch = tile_bytes / box_rows;  // bytes per staged row (2 * min(cols, 256))
+  const int pitch = box_bytes / box_rows;  // bytes per staged row of a box (2 * min(cols, 256))
 
   // Tile t = rb * ncc + cc (rb: 32-row block, counted over all groups; cc:
-  // 256-column chunk).  A CTA visits t = blockIdx.x + k * gridDim.x; the
-  // position advances by (gridDim.x / ncc, gridDim.x % ncc) with a carry and
-  // the group index moves forward with it, so the loop does no 64-bit
-  // division.
+  // column chunk).  A CTA visits t = blockIdx.x + k * gridDim.x; the position
+  // advances by (gridDim.x / ncc, gridDim.x % ncc) with a carry and the group
+  // index moves forward with it, so the loop does no 64-bit division.
   const bool ragged = row_offsets != nullptr;
   const int step_rb = static_cast<int>(gridDim.x) / ncc, step_cc = static_cast<int>(gridDim.x) % ncc;
   struct Pos {
@@ -215,17 +225,6 @@ __global__ void __launch_bounds__(kQThreads, QCfg<kDbias>::kCtasPerSm)
     r0 = gstart + j * kQRows;
     vrows = static_cast<int>(max(int64_t(0), min(static_cast<int64_t>(kQRows), gend - r0)));
   };
-  // Stage s <- the tile at q (rows of other groups and past the tensor are
-  // masked or zero-filled; the consumers use only the block's valid rows).
-  auto issue = [&](const Pos& q, int s) {
-    int64_t jq, rq;
-    int vq;
-    resolve(q, jq, rq, vq);
-    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(tile_bytes));
-    tma_load_2d(stage_buf + s * kQTileBytes, &tm_src, &full[s], q.cc * kQCols, static_cast<int32_t>(rq));
-  };
-
-  int64_t t = blockIdx.x;
   Pos pos;
   pos.rb = static_cast<int>(blockIdx.x) / ncc;
   pos.cc = static_cast<int>(blockIdx.x) % ncc;
@@ -239,186 +238,198 @@ __global__ void __launch_bounds__(kQThreads, QCfg<kDbias>::kCtasPerSm)
     pos.g = lo;
   }
   advance_group(pos);
-  // producer (thread 0): the next tile to load
-  Pos ppos = pos;
-  int64_t ptile = t;
-  int issued = 0, consumed = 0;
-  if (tid == 0) {
-    for (int s = 0; s < kQStages && ptile < ntiles; ++s) {
-      issue(ppos, s);
-      ++issued;
-      ptile += gridDim.x;
-      step(ppos);
+
+  if (warp == kQThreads / 32) {
+    // ===================== producer (one thread) =====================
+    if (lane == 0) {
+      int issued = 0;
+      for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++issued) {
+        const int s = issued % kStages;
+        // the consumers' release of this stage's previous tile
+        if (!mbar_wait(&empty[s], (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, abort_flag)) {
+          if (!*abort_flag) {
+            *abort_flag = 1;
+            if (status != nullptr) atomicOr(status, GL_DEV_TIMEOUT);
+          }
+          break;
+        }
+        int64_t jq, rq;
+        int vq;
+        resolve(pos, jq, rq, vq);
+        // rows of other groups and past the tensor are masked or zero-filled;
+        // the consumers use only the block's valid rows
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kCB * box_bytes));
+#pragma unroll
+        for (int b = 0; b < kCB; ++b)
+          tma_load_2d(stage_buf + s * Q::kTileBytes + b * kQBoxBytes, &tm_src, &full[s],
+                      pos.cc * kTileCols + b * kQCols, static_cast<int32_t>(rq));
+        step(pos);
+      }
+      // never leave while a load may still be writing shared memory
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+      for (int k = issued - kStages > 0 ? issued - kStages : 0; k < issued; ++k)
+        mbar_wait_until(&full[k % kStages], static_cast<uint32_t>(k / kStages) & 1u, deadline);
     }
+    return;
   }
-  for (; t < ntiles; t += gridDim.x, ++consumed) {
-    const int s = consumed % kQStages;
+
+  // ===================== consumers (warps 0-7) =====================
+  const int rg = lane >> 2;   // row group: rows 4 rg .. 4 rg + 3 of the block
+  const int cg = lane & 3;    // 8 columns (16 bytes) of each 32-column block
+  const int rbase = rg * 4;
+  int consumed = 0;
+  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++consumed) {
+    const int s = consumed % kStages;
     const int g = pos.g, cc = pos.cc;
     int64_t j, r0;
     int vrows;
     resolve(pos, j, r0, vrows);
-    // a stage that never lands: flag it, skip the work, leave after the
-    // end-of-tile barrier (every thread reaches it)
-    if (!mbar_wait(&full[s], static_cast<uint32_t>(consumed / kQStages) & 1u, abort_flag)) *abort_flag = 1;
-    const bool work = *abort_flag == 0;
-    // this thread's 4 rows x 8 columns, one 16-byte piece per row (rows past
-    // the block's valid rows read as zero)
-    uint4 raw[4];
-    {
-      const uint8_t* tile = stage_buf + s * kQTileBytes + c8 * 16;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = rbase + i;
-        raw[i] = (work && r < vrows && c8 * 16 < pitch) ? *reinterpret_cast<const uint4*>(tile + r * pitch)
-                                                       : make_uint4(0, 0, 0, 0);
+    if (!mbar_wait(&full[s], static_cast<uint32_t>(consumed / kStages) & 1u, abort_flag)) {
+      if (lane == 0 && !*abort_flag) {
+        *abort_flag = 1;
+        if (status != nullptr) atomicOr(status, GL_DEV_TIMEOUT);
       }
-    }
-    const int col = cc * kQCols + c8 * 8;
-    const bool col_ok = work && col < cols;
-    // |v| as pairs of bf16 bit patterns: for non-negative values the unsigned
-    // order of the bits is the order of the values, so every block maximum
-    // is an integer maximum over 16-bit halves
-    uint32_t mag[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      mag[i][0] = raw[i].x & 0x7FFF7FFFu;
-      mag[i][1] = raw[i].y & 0x7FFF7FFFu;
-      mag[i][2] = raw[i].z & 0x7FFF7FFFu;
-      mag[i][3] = raw[i].w & 0x7FFF7FFFu;
-    }
-    const int64_t tile_off = r0 * cols + col;  // element offset of this thread's first value
-
-    if (codes_r != nullptr) {
-      // row maxima over this thread's 8 columns, two rows per word, then over
-      // the 4 lanes that share each 32-column block
-      uint32_t m[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) m[i] = umax2(umax2(mag[i][0], mag[i][1]), umax2(mag[i][2], mag[i][3]));
-      uint32_t p01 = umax2(__byte_perm(m[0], m[1], 0x5410), __byte_perm(m[0], m[1], 0x7632));
-      uint32_t p23 = umax2(__byte_perm(m[2], m[3], 0x5410), __byte_perm(m[2], m[3], 0x7632));
-      p01 = umax2(p01, __shfl_xor_sync(0xffffffffu, p01, 1));
-      p23 = umax2(p23, __shfl_xor_sync(0xffffffffu, p23, 1));
-      p01 = umax2(p01, __shfl_xor_sync(0xffffffffu, p01, 2));
-      p23 = umax2(p23, __shfl_xor_sync(0xffffffffu, p23, 2));
-      const uint32_t am[4] = {p01 & 0xFFFFu, p01 >> 16, p23 & 0xFFFFu, p23 >> 16};
-      uint8_t* dst = codes_r + tile_off + static_cast<int64_t>(rbase) * cols;
-      uint32_t ebytes = 0;  // biased scale exponents of this thread's 4 rows, row i in byte i
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t byte;
-        const float sc = mx_scale_bf16(am[i], byte);
-        ebytes |= byte << (8 * i);
-        if (col_ok && rbase + i < vrows) *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(raw[i], sc);
-      }
-      // the warp's 4 rows x 8 blocks of 32 columns are 32 scales: lane L
-      // writes the one of row L/8, block L%8 (taken from that block's first
-      // lane), so every lane stores one byte instead of a quarter storing four
-      {
-        const int ri = lane >> 3, blk = lane & 7;
-        const uint32_t eb = __shfl_sync(0xffffffffu, ebytes, blk * 4);
-        const int kb = (cc * kQCols >> 5) + blk;
-        if (work && (kb << 5) < cols && rbase + ri < vrows) {
-          // row-major [rows, cols/32], or the tcgen05 scale-factor atoms:
-          // 512 bytes per (k-group of 4 blocks, 128 rows), row i of the
-          // atom at byte (i%32)*16 + ((i/32)%4)*4 + block
-          const int64_t row = r0 + rbase + ri;
-          const int64_t at = mma_layout ? ((kb >> 2) * mma_rb + (row >> 7)) * 512 +
-                                              static_cast<int>(((row & 31) << 4) | (((row >> 5) & 3) << 2) | (kb & 3))
-                                        : row * (cols >> 5) + kb;
-          scales_r[at] = static_cast<uint8_t>(eb >> (8 * ri));
-        }
-      }
-    }
-
-    // bias gradient: this thread's 4 rows per column (rows past the block's
-    // valid rows were loaded as zeros), published with the next barrier
-    if (kDbias) {
-      float cs[8];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t w0 = (&raw[0].x)[k], w1 = (&raw[1].x)[k], w2 = (&raw[2].x)[k], w3 = (&raw[3].x)[k];
-        cs[2 * k] = ((bf16_lo(w0) + bf16_lo(w1)) + bf16_lo(w2)) + bf16_lo(w3);
-        cs[2 * k + 1] = ((bf16_hi(w0) + bf16_hi(w1)) + bf16_hi(w2)) + bf16_hi(w3);
-      }
-      float4* cp = reinterpret_cast<float4*>(&csum[warp][c8 * 8]);
-      cp[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
-      cp[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
-    }
-    // thread tid: column cc*256 + tid of this block, the 8 warps in order
-    auto store_partial = [&]() {
-      float a = csum[0][tid];
-#pragma unroll
-      for (int w = 1; w < kQThreads / 32; ++w) a += csum[w][tid];
-      const int ccol = cc * kQCols + tid;
-      if (work && ccol < cols && pos.rb < part_blocks) part[pos.rb * cols + ccol] = a;
-    };
-
-    if (codes_c != nullptr) {
-      // column maxima over this thread's 4 rows (two columns per word), then
-      // over the 8 warps through shared memory: thread t < 128 finishes
-      // columns 2t and 2t + 1 of the tile
-      uint4 cm;
-      cm.x = umax2(umax2(mag[0][0], mag[1][0]), umax2(mag[2][0], mag[3][0]));
-      cm.y = umax2(umax2(mag[0][1], mag[1][1]), umax2(mag[2][1], mag[3][1]));
-      cm.z = umax2(umax2(mag[0][2], mag[1][2]), umax2(mag[2][2], mag[3][2]));
-      cm.w = umax2(umax2(mag[0][3], mag[1][3]), umax2(mag[2][3], mag[3][3]));
-      reinterpret_cast<uint4*>(cmax[warp])[c8] = cm;
-      __syncthreads();
-      if (tid < kQCols / 2) {
-        uint32_t a = cmax[0][tid];
-#pragma unroll
-        for (int w = 1; w < kQThreads / 32; ++w) a = umax2(a, cmax[w][tid]);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t byte;
-          csf[2 * tid + h] = mx_scale_bf16(h ? (a >> 16) : (a & 0xFFFFu), byte);
-          const int ccol = cc * kQCols + 2 * tid + h;
-          if (work && ccol < cols && vrows > 0) {
-            int64_t at;
-            if (mma_layout) {
-              // atom (k-group of the group's blocks 4t..4t+3, 128 columns)
-              const int64_t kq = (ragged ? qprefix[g] : static_cast<int64_t>(g) * qpg) + (j >> 2);
-              at = (kq * mma_cb + (ccol >> 7)) * 512 + (((ccol & 31) << 4) | (((ccol >> 5) & 3) << 2) | (j & 3));
-            } else {
-              at = ((ragged ? bprefix[g] : static_cast<int64_t>(g) * bpg) + j) * cols + ccol;
-            }
-            // offsets that overlap (only possible without a status word) must
-            // not push a write past the documented allocation
-            if (at < scales_c_bytes) scales_c[at] = static_cast<uint8_t>(byte);
-          }
-        }
-      }
-      if (kDbias) store_partial();  // csum complete since the barrier above
-      __syncthreads();
-      const float4 s0 = reinterpret_cast<const float4*>(csf)[c8 * 2];
-      const float4 s1 = reinterpret_cast<const float4*>(csf)[c8 * 2 + 1];
-      uint8_t* dst = codes_c + tile_off + static_cast<int64_t>(rbase) * cols;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (col_ok && rbase + i < vrows) *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(raw[i], s0, s1);
-      }
-    }
-    if (kDbias && codes_c == nullptr) {
-      __syncthreads();  // csum complete
-      store_partial();
-    }
-    // every thread is done with stage s (and with cmax / csf / csum): refill it
-    __syncthreads();
-    if (*abort_flag) {
-      if (tid == 0 && status != nullptr) atomicOr(status, GL_DEV_TIMEOUT);
       break;
     }
-    if (tid == 0 && ptile < ntiles) {
-      issue(ppos, s);
-      ++issued;
-      ptile += gridDim.x;
-      step(ppos);
+#pragma unroll
+    for (int b = 0; b < kCB; ++b) {
+      const int cblk = cc * (kTileCols / 32) + b * 8 + warp;  // 32-column block of the tensor
+      const int col = cblk * 32 + cg * 8;                      // this lane's first column
+      const bool col_ok = col < cols;
+      // this lane's 4 rows x 8 columns, one 16-byte piece per row (rows past
+      // the block's valid rows and columns past the tensor read as zero)
+      uint4 raw[4];
+      {
+        const uint8_t* tile = stage_buf + s * Q::kTileBytes + b * kQBoxBytes + (warp * 32 + cg * 8) * 2;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = rbase + i;
+          raw[i] = (r < vrows && col_ok) ? *reinterpret_cast<const uint4*>(tile + r * pitch) : make_uint4(0, 0, 0, 0);
+        }
+      }
+      // |v| as pairs of bf16 bit patterns: for non-negative values the
+      // unsigned order of the bits is the order of the values, so every
+      // block maximum is an integer maximum over 16-bit halves
+      uint32_t mag[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mag[i][0] = raw[i].x & 0x7FFF7FFFu;
+        mag[i][1] = raw[i].y & 0x7FFF7FFFu;
+        mag[i][2] = raw[i].z & 0x7FFF7FFFu;
+        mag[i][3] = raw[i].w & 0x7FFF7FFFu;
+      }
+      const int64_t tile_off = r0 * cols + col;  // element offset of this lane's first value
+
+      if (codes_r != nullptr) {
+        // row maxima over this lane's 8 columns, two rows per word, then over
+        // the 4 lanes of the row group (lane bits 0-1)
+        uint32_t m[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m[i] = umax2(umax2(mag[i][0], mag[i][1]), umax2(mag[i][2], mag[i][3]));
+        uint32_t p01 = umax2(__byte_perm(m[0], m[1], 0x5410), __byte_perm(m[0], m[1], 0x7632));
+        uint32_t p23 = umax2(__byte_perm(m[2], m[3], 0x5410), __byte_perm(m[2], m[3], 0x7632));
+        p01 = umax2(p01, __shfl_xor_sync(0xffffffffu, p01, 1));
+        p23 = umax2(p23, __shfl_xor_sync(0xffffffffu, p23, 1));
+        p01 = umax2(p01, __shfl_xor_sync(0xffffffffu, p01, 2));
+        p23 = umax2(p23, __shfl_xor_sync(0xffffffffu, p23, 2));
+        const uint32_t am[4] = {p01 & 0xFFFFu, p01 >> 16, p23 & 0xFFFFu, p23 >> 16};
+        uint8_t* dst = codes_r + tile_off + static_cast<int64_t>(rbase) * cols;
+        uint32_t ebytes = 0;  // biased scale exponents of the 4 rows, row i in byte i
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t byte;
+          const float sc = mx_scale_bf16(am[i], byte);
+          ebytes |= byte << (8 * i);
+          if (col_ok && rbase + i < vrows) *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(raw[i], sc);
+        }
+        // the row group's 4 scales: lane cg stores the one of row rbase + cg
+        if ((cblk << 5) < cols && rbase + cg < vrows) {
+          // row-major [rows, cols/32], or the tcgen05 scale-factor atoms: 512
+          // bytes per (k-group of 4 blocks, 128 rows), row i of the atom at
+          // byte (i%32)*16 + ((i/32)%4)*4 + block
+          const int64_t row = r0 + rbase + cg;
+          const int64_t at = mma_layout ? ((cblk >> 2) * mma_rb + (row >> 7)) * 512 +
+                                              static_cast<int>(((row & 31) << 4) | (((row >> 5) & 3) << 2) | (cblk & 3))
+                                        : row * (cols >> 5) + cblk;
+          scales_r[at] = static_cast<uint8_t>(ebytes >> (8 * cg));
+        }
+      }
+
+      if (codes_c != nullptr) {
+        // column maxima over this lane's 4 rows (two columns per word), then
+        // over the 8 row groups (lane bits 2-4)
+        uint32_t cm[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          cm[k] = umax2(umax2(mag[0][k], mag[1][k]), umax2(mag[2][k], mag[3][k]));
+          cm[k] = umax2(cm[k], __shfl_xor_sync(0xffffffffu, cm[k], 4));
+          cm[k] = umax2(cm[k], __shfl_xor_sync(0xffffffffu, cm[k], 8));
+          cm[k] = umax2(cm[k], __shfl_xor_sync(0xffffffffu, cm[k], 16));
+        }
+        float sc[8];
+        uint32_t cb_lo = 0, cb_hi = 0;  // biased exponents of columns 0-3 / 4-7, column i in byte i % 4
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t b0, b1;
+          sc[2 * k] = mx_scale_bf16(cm[k] & 0xFFFFu, b0);
+          sc[2 * k + 1] = mx_scale_bf16(cm[k] >> 16, b1);
+          const uint32_t two = b0 | (b1 << 8);
+          if (k < 2) cb_lo |= two << (16 * k);
+          else       cb_hi |= two << (16 * (k - 2));
+        }
+        const float4 s0 = make_float4(sc[0], sc[1], sc[2], sc[3]);
+        const float4 s1 = make_float4(sc[4], sc[5], sc[6], sc[7]);
+        uint8_t* dst = codes_c + tile_off + static_cast<int64_t>(rbase) * cols;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (col_ok && rbase + i < vrows) *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(raw[i], s0, s1);
+        // the 8 columns' scales: lane rg stores the one of column col + rg
+        const int ccol = col + rg;
+        if (ccol < cols && vrows > 0) {
+          int64_t at;
+          if (mma_layout) {
+            // atom (k-group of the group's blocks 4t..4t+3, 128 columns)
+            const int64_t kq = (ragged ? qprefix[g] : static_cast<int64_t>(g) * qpg) + (j >> 2);
+            at = (kq * mma_cb + (ccol >> 7)) * 512 + (((ccol & 31) << 4) | (((ccol >> 5) & 3) << 2) | (j & 3));
+          } else {
+            at = ((ragged ? bprefix[g] : static_cast<int64_t>(g) * bpg) + j) * cols + ccol;
+          }
+          // offsets that overlap (only possible without a status word) must
+          // not push a write past the documented allocation
+          if (at < scales_c_bytes) scales_c[at] = static_cast<uint8_t>((rg < 4 ? cb_lo : cb_hi) >> (8 * (rg & 3)));
+        }
+      }
+
+      if (kDbias) {
+        // bias gradient: this lane's 4 rows per column (rows past the block's
+        // valid rows were loaded as zeros), then the 8 row groups by a
+        // butterfly (every lane ends with the same sums); lane rg stores
+        // column col + rg
+        float cs[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t w0 = (&raw[0].x)[k], w1 = (&raw[1].x)[k], w2 = (&raw[2].x)[k], w3 = (&raw[3].x)[k];
+          cs[2 * k] = ((bf16_lo(w0) + bf16_lo(w1)) + bf16_lo(w2)) + bf16_lo(w3);
+          cs[2 * k + 1] = ((bf16_hi(w0) + bf16_hi(w1)) + bf16_hi(w2)) + bf16_hi(w3);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 4);
+          cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 8);
+          cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 16);
+        }
+        float mine = cs[0];
+#pragma unroll
+        for (int k = 1; k < 8; ++k)
+          if (rg == k) mine = cs[k];
+        const int ccol = col + rg;
+        if (ccol < cols && pos.rb < part_blocks) part[pos.rb * cols + ccol] = mine;
+      }
     }
+    // this warp is done with stage s
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
     step(pos);
-  }
-  if (tid == 0) {
-    // never leave while a load may still be writing shared memory
-    for (int k2 = consumed; k2 < issued; ++k2) mbar_wait_bounded(&full[k2 % kQStages], (k2 / kQStages) & 1);
   }
 }
 
@@ -438,24 +449,28 @@ gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t
   if (!encode_tmap(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, src, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
     return GL_ERR_UNSUPPORTED;
   const int prefix_bytes = row_offsets != nullptr ? 2 * (G + 1) * static_cast<int>(sizeof(int64_t)) : 0;
-  const int tile_bytes = static_cast<int>(box_cols * box_rows * 2);
+  const int box_bytes = static_cast<int>(box_cols * box_rows * 2);
   const int64_t sc_bytes = static_cast<int64_t>(gl_mxfp8_scale_bytes(rows, cols, G, 1, scale_layout));
   const int mma = scale_layout == GL_SCALES_MMA ? 1 : 0;
+  auto run = [&](auto kern, int stages, int tile_bytes, int ctas_per_sm, float* pt, int64_t pb, int64_t* pp) {
+    const int smem = 1024 + stages * tile_bytes + 128 + prefix_bytes;
+    if (set_max_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return GL_ERR_CUDA;
+    kern<<<num_sms() * ctas_per_sm, kQThreads + 32, smem, stream>>>(
+        tm, rows, cols, static_cast<int>(box_rows), box_bytes, row_offsets, G, status, codes_r, scales_r, codes_c,
+        scales_c, sc_bytes, mma, pt, pb, pp);
+    return GL_OK;
+  };
+  // two boxes per tile once the rows are wider than one box
+  const bool wide = cols > kQCols;
+  gl_status st;
   if (part != nullptr) {
-    using Q = QCfg<true>;
-    const int smem = 1024 + Q::kStages * kQTileBytes + 64 + prefix_bytes;
-    if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel<true>), smem) != cudaSuccess) return GL_ERR_CUDA;
-    quantize_kernel<true><<<num_sms() * Q::kCtasPerSm, kQThreads, smem, stream>>>(
-        tm, rows, cols, static_cast<int>(box_rows), tile_bytes, row_offsets, G, status, codes_r, scales_r, codes_c,
-        scales_c, sc_bytes, mma, part, part_blocks, part_prefix);
+    if (wide) st = run(quantize_kernel<true, 2>, QCfg<true, 2>::kStages, QCfg<true, 2>::kTileBytes, QCfg<true, 2>::kCtasPerSm, part, part_blocks, part_prefix);
+    else      st = run(quantize_kernel<true, 1>, QCfg<true, 1>::kStages, QCfg<true, 1>::kTileBytes, QCfg<true, 1>::kCtasPerSm, part, part_blocks, part_prefix);
   } else {
-    using Q = QCfg<false>;
-    const int smem = 1024 + Q::kStages * kQTileBytes + 64 + prefix_bytes;
-    if (set_max_smem(reinterpret_cast<const void*>(quantize_kernel<false>), smem) != cudaSuccess) return GL_ERR_CUDA;
-    quantize_kernel<false><<<num_sms() * Q::kCtasPerSm, kQThreads, smem, stream>>>(
-        tm, rows, cols, static_cast<int>(box_rows), tile_bytes, row_offsets, G, status, codes_r, scales_r, codes_c,
-        scales_c, sc_bytes, mma, nullptr, 0, nullptr);
+    if (wide) st = run(quantize_kernel<false, 2>, QCfg<false, 2>::kStages, QCfg<false, 2>::kTileBytes, QCfg<false, 2>::kCtasPerSm, nullptr, 0, nullptr);
+    else      st = run(quantize_kernel<false, 1>, QCfg<false, 1>::kStages, QCfg<false, 1>::kTileBytes, QCfg<false, 1>::kCtasPerSm, nullptr, 0, nullptr);
   }
+  if (st != GL_OK) return st;
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
 }
 
