@@ -42,7 +42,7 @@ namespace {
 constexpr int BK = 64;  // contraction elements of a K-major stage (one 128-byte swizzle row)
 constexpr int kPG = 64;  // per-group tensor maps carried by one launch
 constexpr int kSmemBudget = 212992;  // stage ring (pairs: 3 x 64 KB; single CTAs: 4 x 48 KB) + (wgrad) 16 KB of transposes
-constexpr int kBand = 8;  // tile rows per rasterisation band
+constexpr int kBand = 16;  // tile rows per rasterisation band
 
 template <int MODE, int CG>
 struct Cfg {

@@ -48,7 +48,7 @@ namespace {
 
 constexpr int BK = 128;  // fp8 contraction elements per sub-stage (128 bytes: one swizzle row, one scale k-group)
 constexpr int kPG = 64;
-constexpr int kBand = 8;
+constexpr int kBand = 16;  // tile rows per rasterisation band
 constexpr int kSfSlots = 4;      // slot j: A at +0 (4 columns), B at +4 (8 columns)
 constexpr int kSfSlotCols = 16;
 constexpr int kSfABytes = 512;   // one atom
