@@ -42,7 +42,12 @@ namespace {
 constexpr int BK = 64;  // contraction elements of a K-major stage (one 128-byte swizzle row)
 constexpr int kPG = 64;  // per-group tensor maps carried by one launch
 constexpr int kSmemBudget = 212992;  // stage ring (pairs: 3 x 64 KB; single CTAs: 4 x 48 KB) + (wgrad) 16 KB of transposes
-constexpr int kBand = 16;  // tile rows per rasterisation band
+// Tile rows per rasterisation band: 16 for fwd (a band's A strips, 16 x 256
+// rows of x, stay in L2 while the band sweeps W, which it reads once);
+// dgrad's A strips span the whole N contraction (3.5x longer at the
+// 14336-wide layer), so it keeps 8, as does wgrad (no measured difference).
+template <int MODE>
+__host__ __device__ constexpr int band_rows() { return MODE == kFwd ? 16 : 8; }
 
 template <int MODE, int CG>
 struct Cfg {
@@ -149,6 +154,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const Gemm
   // near-square block and share operand strips through L2.
   const int mtg = (MODE == kWgrad) ? ceil_div_i(p.N, C::kTileM) : ceil_div_i(m, C::kTileM);
   const int ntg = ceil_div_i(MODE == kFwd ? p.N : p.K, C::kTileN);
+  constexpr int kBand = band_rows<MODE>();
   const int band = local / (kBand * ntg);
   const int base_mt = band * kBand;
   const int bh = min(kBand, mtg - base_mt);

@@ -47,7 +47,7 @@ template <bool kDbias, int kCB>
 struct QCfg {
   static constexpr int kTileBytes = kCB * kQBoxBytes;
   static constexpr int kStages = kCB == 1 ? 4 : 3;
-  static constexpr int kCtasPerSm = kCB == 1 ? 3 : 2;
+  static constexpr int kCtasPerSm = 2;
 };
 
 // Per 16-bit half: the unsigned maximum.
@@ -74,39 +74,26 @@ __device__ __forceinline__ float mx_scale_bf16(uint32_t a, uint32_t& byte) {
   return __uint_as_float(a ? (262u - ec) << 23 : 0x3F800000u);
 }
 
-// (a, b) * (sa, sb) with one packed fp32 multiply (exact here: the scales
-// are powers of two and the products stay in the normal range or round to
-// zero in E4M3 anyway), rounded to two E4M3 codes (satfinite), a in the low
-// byte.
-__device__ __forceinline__ uint32_t e4m3x2_scaled(float a, float b, float sa, float sb) {
-  uint16_t q;
-  asm("{\n\t.reg .b64 v, s, p;\n\t.reg .f32 x, y;\n\t"
-      "mov.b64 v, {%1, %2};\n\t"
-      "mov.b64 s, {%3, %4};\n\t"
-      "mul.rn.f32x2 p, v, s;\n\t"
-      "mov.b64 {x, y}, p;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 %0, y, x;\n\t}"
-      : "=h"(q)
-      : "f"(a), "f"(b), "f"(sa), "f"(sb));
-  return q;
-}
-
-// Eight bf16 values (four words, first value lowest) times one scale ->
-// eight E4M3 codes.
-__device__ __forceinline__ uint2 e4m3x8(const uint4& w, float sc) {
-  uint2 q;
-  q.x = e4m3x2_scaled(bf16_lo(w.x), bf16_hi(w.x), sc, sc) | (e4m3x2_scaled(bf16_lo(w.y), bf16_hi(w.y), sc, sc) << 16);
-  q.y = e4m3x2_scaled(bf16_lo(w.z), bf16_hi(w.z), sc, sc) | (e4m3x2_scaled(bf16_lo(w.w), bf16_hi(w.w), sc, sc) << 16);
-  return q;
-}
-
-// Same, value j scaled by its column's scale (s0: columns 0-3, s1: 4-7).
-__device__ __forceinline__ uint2 e4m3x8(const uint4& w, const float4& s0, const float4& s1) {
-  uint2 q;
-  q.x = e4m3x2_scaled(bf16_lo(w.x), bf16_hi(w.x), s0.x, s0.y) |
-        (e4m3x2_scaled(bf16_lo(w.y), bf16_hi(w.y), s0.z, s0.w) << 16);
-  q.y = e4m3x2_scaled(bf16_lo(w.z), bf16_hi(w.z), s1.x, s1.y) |
-        (e4m3x2_scaled(bf16_lo(w.w), bf16_hi(w.w), s1.z, s1.w) << 16);
+// Four values times their scales (exact: powers of two; two packed fp32
+// multiplies), rounded to four E4M3 codes (satfinite), the first value in the
+// lowest byte.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d, float sa, float sb, float sc,
+                                           float sd) {
+  uint32_t q;
+  asm("{\n\t.reg .b64 v0, v1, s0, s1, p0, p1;\n\t.reg .f32 x0, y0, x1, y1;\n\t.reg .b16 l, h;\n\t"
+      "mov.b64 v0, {%1, %2};\n\t"
+      "mov.b64 v1, {%3, %4};\n\t"
+      "mov.b64 s0, {%5, %6};\n\t"
+      "mov.b64 s1, {%7, %8};\n\t"
+      "mul.rn.f32x2 p0, v0, s0;\n\t"
+      "mul.rn.f32x2 p1, v1, s1;\n\t"
+      "mov.b64 {x0, y0}, p0;\n\t"
+      "mov.b64 {x1, y1}, p1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 l, y0, x0;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h, y1, x1;\n\t"
+      "mov.b32 %0, {l, h};\n\t}"
+      : "=r"(q)
+      : "f"(a), "f"(b), "f"(c), "f"(d), "f"(sa), "f"(sb), "f"(sc), "f"(sd));
   return q;
 }
 
@@ -320,9 +307,15 @@ __global__ void __launch_bounds__(kQThreads + 32, QCfg<kDbias, kCB>::kCtasPerSm)
       }
       const int64_t tile_off = r0 * cols + col;  // element offset of this lane's first value
 
+      // Block maxima.  Rows: over this lane's 8 columns, two rows per word,
+      // then over the 4 lanes of the row group (lane bits 0-1).  Columns: over
+      // this lane's 4 rows (two columns per word), then over the 8 row groups
+      // (lane bits 2-4).  Every lane ends with the maxima of all its rows and
+      // columns; it turns one of each into a scale (row rbase + cg, column
+      // col + rg) and the others arrive by shuffles.
+      float rs[4], cs[8];
+      uint32_t rbyte = 0, cbyte = 0;
       if (codes_r != nullptr) {
-        // row maxima over this lane's 8 columns, two rows per word, then over
-        // the 4 lanes of the row group (lane bits 0-1)
         uint32_t m[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) m[i] = umax2(umax2(mag[i][0], mag[i][1]), umax2(mag[i][2], mag[i][3]));
@@ -332,32 +325,12 @@ __global__ void __launch_bounds__(kQThreads + 32, QCfg<kDbias, kCB>::kCtasPerSm)
         p23 = umax2(p23, __shfl_xor_sync(0xffffffffu, p23, 1));
         p01 = umax2(p01, __shfl_xor_sync(0xffffffffu, p01, 2));
         p23 = umax2(p23, __shfl_xor_sync(0xffffffffu, p23, 2));
-        const uint32_t am[4] = {p01 & 0xFFFFu, p01 >> 16, p23 & 0xFFFFu, p23 >> 16};
-        uint8_t* dst = codes_r + tile_off + static_cast<int64_t>(rbase) * cols;
-        uint32_t ebytes = 0;  // biased scale exponents of the 4 rows, row i in byte i
+        const uint32_t pw = (cg & 2) ? p23 : p01;
+        const float own = mx_scale_bf16((cg & 1) ? (pw >> 16) : (pw & 0xFFFFu), rbyte);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t byte;
-          const float sc = mx_scale_bf16(am[i], byte);
-          ebytes |= byte << (8 * i);
-          if (col_ok && rbase + i < vrows) *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(raw[i], sc);
-        }
-        // the row group's 4 scales: lane cg stores the one of row rbase + cg
-        if ((cblk << 5) < cols && rbase + cg < vrows) {
-          // row-major [rows, cols/32], or the tcgen05 scale-factor atoms: 512
-          // bytes per (k-group of 4 blocks, 128 rows), row i of the atom at
-          // byte (i%32)*16 + ((i/32)%4)*4 + block
-          const int64_t row = r0 + rbase + cg;
-          const int64_t at = mma_layout ? ((cblk >> 2) * mma_rb + (row >> 7)) * 512 +
-                                              static_cast<int>(((row & 31) << 4) | (((row >> 5) & 3) << 2) | (cblk & 3))
-                                        : row * (cols >> 5) + cblk;
-          scales_r[at] = static_cast<uint8_t>(ebytes >> (8 * cg));
-        }
+        for (int i = 0; i < 4; ++i) rs[i] = __shfl_sync(0xffffffffu, own, (lane & ~3) | i);
       }
-
       if (codes_c != nullptr) {
-        // column maxima over this lane's 4 rows (two columns per word), then
-        // over the 8 row groups (lane bits 2-4)
         uint32_t cm[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -366,24 +339,47 @@ __global__ void __launch_bounds__(kQThreads + 32, QCfg<kDbias, kCB>::kCtasPerSm)
           cm[k] = umax2(cm[k], __shfl_xor_sync(0xffffffffu, cm[k], 8));
           cm[k] = umax2(cm[k], __shfl_xor_sync(0xffffffffu, cm[k], 16));
         }
-        float sc[8];
-        uint32_t cb_lo = 0, cb_hi = 0;  // biased exponents of columns 0-3 / 4-7, column i in byte i % 4
+        const uint32_t cw = (rg & 4) ? ((rg & 2) ? cm[3] : cm[2]) : ((rg & 2) ? cm[1] : cm[0]);
+        const float own = mx_scale_bf16((rg & 1) ? (cw >> 16) : (cw & 0xFFFFu), cbyte);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t b0, b1;
-          sc[2 * k] = mx_scale_bf16(cm[k] & 0xFFFFu, b0);
-          sc[2 * k + 1] = mx_scale_bf16(cm[k] >> 16, b1);
-          const uint32_t two = b0 | (b1 << 8);
-          if (k < 2) cb_lo |= two << (16 * k);
-          else       cb_hi |= two << (16 * (k - 2));
+        for (int k = 0; k < 8; ++k) cs[k] = __shfl_sync(0xffffffffu, own, (k << 2) | cg);
+      }
+
+      // codes: each row unpacked once, then scaled and rounded for each copy
+      {
+        uint8_t* dr = (codes_r != nullptr) ? codes_r + tile_off + static_cast<int64_t>(rbase) * cols : nullptr;
+        uint8_t* dc = (codes_c != nullptr) ? codes_c + tile_off + static_cast<int64_t>(rbase) * cols : nullptr;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (!(col_ok && rbase + i < vrows)) continue;
+          float f[8];
+          f[0] = bf16_lo(raw[i].x); f[1] = bf16_hi(raw[i].x);
+          f[2] = bf16_lo(raw[i].y); f[3] = bf16_hi(raw[i].y);
+          f[4] = bf16_lo(raw[i].z); f[5] = bf16_hi(raw[i].z);
+          f[6] = bf16_lo(raw[i].w); f[7] = bf16_hi(raw[i].w);
+          if (codes_r != nullptr)
+            *reinterpret_cast<uint2*>(dr + i * cols) =
+                make_uint2(e4m3x4(f[0], f[1], f[2], f[3], rs[i], rs[i], rs[i], rs[i]),
+                           e4m3x4(f[4], f[5], f[6], f[7], rs[i], rs[i], rs[i], rs[i]));
+          if (codes_c != nullptr)
+            *reinterpret_cast<uint2*>(dc + i * cols) =
+                make_uint2(e4m3x4(f[0], f[1], f[2], f[3], cs[0], cs[1], cs[2], cs[3]),
+                           e4m3x4(f[4], f[5], f[6], f[7], cs[4], cs[5], cs[6], cs[7]));
         }
-        const float4 s0 = make_float4(sc[0], sc[1], sc[2], sc[3]);
-        const float4 s1 = make_float4(sc[4], sc[5], sc[6], sc[7]);
-        uint8_t* dst = codes_c + tile_off + static_cast<int64_t>(rbase) * cols;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (col_ok && rbase + i < vrows) *reinterpret_cast<uint2*>(dst + i * cols) = e4m3x8(raw[i], s0, s1);
-        // the 8 columns' scales: lane rg stores the one of column col + rg
+      }
+
+      // scale bytes: this lane's row and column
+      if (codes_r != nullptr && (cblk << 5) < cols && rbase + cg < vrows) {
+        // row-major [rows, cols/32], or the tcgen05 scale-factor atoms: 512
+        // bytes per (k-group of 4 blocks, 128 rows), row i of the atom at
+        // byte (i%32)*16 + ((i/32)%4)*4 + block
+        const int64_t row = r0 + rbase + cg;
+        const int64_t at = mma_layout ? ((cblk >> 2) * mma_rb + (row >> 7)) * 512 +
+                                            static_cast<int>(((row & 31) << 4) | (((row >> 5) & 3) << 2) | (cblk & 3))
+                                      : row * (cols >> 5) + cblk;
+        scales_r[at] = static_cast<uint8_t>(rbyte);
+      }
+      if (codes_c != nullptr) {
         const int ccol = col + rg;
         if (ccol < cols && vrows > 0) {
           int64_t at;
@@ -396,7 +392,7 @@ __global__ void __launch_bounds__(kQThreads + 32, QCfg<kDbias, kCB>::kCtasPerSm)
           }
           // offsets that overlap (only possible without a status word) must
           // not push a write past the documented allocation
-          if (at < scales_c_bytes) scales_c[at] = static_cast<uint8_t>((rg < 4 ? cb_lo : cb_hi) >> (8 * (rg & 3)));
+          if (at < scales_c_bytes) scales_c[at] = static_cast<uint8_t>(cbyte);
         }
       }
 
