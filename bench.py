@@ -50,12 +50,17 @@ OP_SAMPLES = 50  # per-op medians are taken over at least this many steps
 # of the CUDA sources the capture ran.  When the sources have changed since,
 # the figures describe other kernels: the line then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "csrc_digest": "e370edcf86e2e803",
+    "csrc_digest": "e74bd1d6ced08fba",
     # the second step of `bench.py --steps 2 --warmup 3` under ncu (one pass,
     # gpu__time_duration / dram__bytes_read / dram__bytes_write per launch)
-    "bf16_g8": {"fwd": 2156613632, "dgrad": 2842237696, "wgrad": 5757256960,
-                "quant_x": 218416896, "quant_w": 1888783616, "quant_dy": 930946048,
-                "fwd_mx": 1206449152, "dgrad_mx": 1418826752, "wgrad_mx": 3658960640},
+    "bf16_g8": {"fwd": 2145088000, "dgrad": 3269915392, "wgrad": 5749022976,
+                "quant_x": 219430144, "quant_w": 1877936896, "quant_dy": 914457344,
+                "fwd_mx": 1011228416, "dgrad_mx": 1386709504, "wgrad_mx": 3693348096},
+    # `bench.py --workload stacked_g128_ragged --steps 1 --warmup 1` under ncu
+    # (the timed step's kernels; the MXFP8 wgrad from the warm-up step)
+    "stacked_g128_ragged": {"fwd": 6160489984, "dgrad": 4638518272, "wgrad": 15695026176,
+                            "quant_x": 1889473280, "quant_w": 7875813632, "quant_dy": 494323968,
+                            "fwd_mx": 2900109824, "dgrad_mx": 2829066496, "wgrad_mx": 14988268032},
 }
 
 
