@@ -18,15 +18,15 @@
 // reductions (each tile's main_grad rows first pulled into L2 with bulk
 // prefetches).  The remaining TMEM columns hold the scale-factor slots.
 //
-// Per stage (128 contraction elements = four MMAs of K=32) the producer
-// TMA-loads the codes (128-byte swizzle) and the scales.  The scales arrive
-// from the quantizer in 512-byte atoms that already have the tcgen05
-// scale-factor layout (128 operand rows x 4 blocks; row i at byte
-// (i%32)*16 + ((i/32)%4)*4 + block), so a stage's scales are two plain boxes:
-// one atom for the CTA's 128 A rows and two consecutive atoms (256 rows)
-// covering the tile's B rows.  The MMA thread copies them to TMEM with
-// tcgen05.cp.32x128b.warpx4 and selects scale byte kb of each MMA through the
-// instruction descriptor.  A tiles (fprop / dgrad) start on 128-row
+// Per sub-stage (128 contraction elements = four MMAs of K=32; a stage holds
+// two on CTA pairs for fprop / dgrad, one otherwise) the producer TMA-loads
+// the codes (128-byte swizzle) and the scales.  The scales arrive from the
+// quantizer in 512-byte atoms that already have the tcgen05 scale-factor
+// layout (128 operand rows x 4 blocks; row i at byte (i%32)*16 + ((i/32)%4)*4
+// + block), so a sub-stage's scales are two plain boxes: one atom for the
+// CTA's 128 A rows and two consecutive atoms (256 rows) covering the tile's B
+// rows.  The MMA thread copies them to TMEM with tcgen05.cp.32x128b.warpx4
+// and selects scale byte kb of each MMA through the instruction descriptor.  A tiles (fprop / dgrad) start on 128-row
 // boundaries of the packed activations: a group's first tile may begin inside
 // the previous group, and only the group's own rows are stored.
 //

@@ -43,7 +43,7 @@ static_assert(kQThreads == 256 && kQCols == 256, "eight consumer warps, one 32-c
 // Tiles staged in shared memory by TMA, and CTAs per SM (each CTA: eight
 // consumer warps and a producer warp).
 constexpr int kQBoxBytes = kQRows * kQCols * 2;  // one TMA box: 32 rows x 256 columns
-template <bool kDbias, int kCB>
+template <int kCB>
 struct QCfg {
   static constexpr int kTileBytes = kCB * kQBoxBytes;
   static constexpr int kStages = kCB == 1 ? 4 : 3;
@@ -110,14 +110,14 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d, f
 // fp32, block b of the launch in row b; part_prefix: the groups' first
 // blocks, int64[G+1], written by CTA 0).
 template <bool kDbias, int kCB>
-__global__ void __launch_bounds__(kQThreads + 32, QCfg<kDbias, kCB>::kCtasPerSm)
+__global__ void __launch_bounds__(kQThreads + 32, QCfg<kCB>::kCtasPerSm)
     quantize_kernel(const __grid_constant__ CUtensorMap tm_src, int64_t rows, int cols, int box_rows,
                     int box_bytes, const int64_t* __restrict__ row_offsets, int G, int32_t* status,
                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r,
                     uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, int64_t scales_c_bytes,
                     int mma_layout, float* __restrict__ part, int64_t part_blocks,
                     int64_t* __restrict__ part_prefix) {
-  using Q = QCfg<kDbias, kCB>;
+  using Q = QCfg<kCB>;
   constexpr int kStages = Q::kStages;
   constexpr int kTileCols = kCB * kQCols;
   extern __shared__ uint8_t qsmem_raw[];
@@ -460,11 +460,11 @@ gl_status launch_quantize(const void* src, int64_t rows, int cols, const int64_t
   const bool wide = cols > kQCols;
   gl_status st;
   if (part != nullptr) {
-    if (wide) st = run(quantize_kernel<true, 2>, QCfg<true, 2>::kStages, QCfg<true, 2>::kTileBytes, QCfg<true, 2>::kCtasPerSm, part, part_blocks, part_prefix);
-    else      st = run(quantize_kernel<true, 1>, QCfg<true, 1>::kStages, QCfg<true, 1>::kTileBytes, QCfg<true, 1>::kCtasPerSm, part, part_blocks, part_prefix);
+    if (wide) st = run(quantize_kernel<true, 2>, QCfg<2>::kStages, QCfg<2>::kTileBytes, QCfg<2>::kCtasPerSm, part, part_blocks, part_prefix);
+    else      st = run(quantize_kernel<true, 1>, QCfg<1>::kStages, QCfg<1>::kTileBytes, QCfg<1>::kCtasPerSm, part, part_blocks, part_prefix);
   } else {
-    if (wide) st = run(quantize_kernel<false, 2>, QCfg<false, 2>::kStages, QCfg<false, 2>::kTileBytes, QCfg<false, 2>::kCtasPerSm, nullptr, 0, nullptr);
-    else      st = run(quantize_kernel<false, 1>, QCfg<false, 1>::kStages, QCfg<false, 1>::kTileBytes, QCfg<false, 1>::kCtasPerSm, nullptr, 0, nullptr);
+    if (wide) st = run(quantize_kernel<false, 2>, QCfg<2>::kStages, QCfg<2>::kTileBytes, QCfg<2>::kCtasPerSm, nullptr, 0, nullptr);
+    else      st = run(quantize_kernel<false, 1>, QCfg<1>::kStages, QCfg<1>::kTileBytes, QCfg<1>::kCtasPerSm, nullptr, 0, nullptr);
   }
   if (st != GL_OK) return st;
   return cudaGetLastError() == cudaSuccess ? GL_OK : GL_ERR_CUDA;
