@@ -50,17 +50,17 @@ OP_SAMPLES = 50  # per-op medians are taken over at least this many steps
 # of the CUDA sources the capture ran.  When the sources have changed since,
 # the figures describe other kernels: the line then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "csrc_digest": "e74bd1d6ced08fba",
+    "csrc_digest": "9ce8bc2146b2dc9f",
     # the second step of `bench.py --steps 2 --warmup 3` under ncu (one pass,
     # gpu__time_duration / dram__bytes_read / dram__bytes_write per launch)
-    "bf16_g8": {"fwd": 2145088000, "dgrad": 3269915392, "wgrad": 5749022976,
-                "quant_x": 219430144, "quant_w": 1877936896, "quant_dy": 914457344,
-                "fwd_mx": 1011228416, "dgrad_mx": 1386709504, "wgrad_mx": 3693348096},
+    "bf16_g8": {"fwd": 1852200704, "dgrad": 2837817088, "wgrad": 5739353344,
+                "quant_x": 219744000, "quant_w": 1877931008, "quant_dy": 914936576,
+                "fwd_mx": 1006996480, "dgrad_mx": 1392577792, "wgrad_mx": 3656645120},
     # `bench.py --workload stacked_g128_ragged --steps 1 --warmup 1` under ncu
     # (the timed step's kernels; the MXFP8 wgrad from the warm-up step)
-    "stacked_g128_ragged": {"fwd": 6160489984, "dgrad": 4638518272, "wgrad": 15695026176,
-                            "quant_x": 1889473280, "quant_w": 7875813632, "quant_dy": 494323968,
-                            "fwd_mx": 2900109824, "dgrad_mx": 2829066496, "wgrad_mx": 14988268032},
+    "stacked_g128_ragged": {"fwd": 5775737088, "dgrad": 4620293120, "wgrad": 15831860992,
+                            "quant_x": 1889802496, "quant_w": 7889447680, "quant_dy": 494449920,
+                            "fwd_mx": 2744198144, "dgrad_mx": 2817394432, "wgrad_mx": 14997782528},
 }
 
 
