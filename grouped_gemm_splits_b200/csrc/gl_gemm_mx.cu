@@ -13,13 +13,13 @@
 // One fp32 accumulator (256 TMEM columns) per tile: eight epilogue warps (two
 // per TMEM lane quarter, 128 columns each) copy it to registers and free it
 // at once, so the next tile's MMAs overlap the stores -- fprop / dgrad round
-// to bf16 (+ bias); wgrad transposes 32 x 32 fp32 chunks through shared
+// to bf16 (+ bias); wgrad transposes 32 x 16 fp32 pieces through shared
 // memory and adds them into main_grad with coalesced 16-byte vector
 // reductions (each tile's main_grad rows first pulled into L2 with bulk
 // prefetches).  The remaining TMEM columns hold the scale-factor slots.
 //
 // Per sub-stage (128 contraction elements = four MMAs of K=32; a stage holds
-// two on CTA pairs for fprop / dgrad, one otherwise) the producer TMA-loads
+// two on CTA pairs, one on single CTAs) the producer TMA-loads
 // the codes (128-byte swizzle) and the scales.  The scales arrive from the
 // quantizer in 512-byte atoms that already have the tcgen05 scale-factor
 // layout (128 operand rows x 4 blocks; row i at byte (i%32)*16 + ((i/32)%4)*4
@@ -54,7 +54,8 @@ constexpr int kSfSlotCols = 16;
 constexpr int kSfABytes = 512;   // one atom
 constexpr int kAtomsB = 2;       // the 256 B rows of a tile
 constexpr int kSfBytes = 2048;   // a sub-stage's A atom + B atoms, padded to keep stages 1 KB aligned
-constexpr int kWgradSub = 1;     // sub-stages per wgrad stage on CTA pairs
+constexpr int kWgradSub = 2;     // sub-stages per wgrad stage on CTA pairs
+constexpr int kWgradMaxG = 256;  // groups per wgrad launch (their tile / scale prefixes share the shared memory)
 static_assert(kSfABytes + kAtomsB * 512 <= kSfBytes, "scale staging");
 
 template <int MODE, int CG>
@@ -67,8 +68,10 @@ struct CfgMX {
   static constexpr int kTileM = 128 * CG;
   static constexpr int kBRows = kTN / CG;  // B rows held per CTA
   // A stage holds kSub sub-stages of 128 contraction elements, each with its
-  // own codes and scale atoms: two on CTA pairs for fprop / dgrad (half the
-  // barrier round trips per MMA, ~8% faster), one elsewhere.
+  // own codes and scale atoms: two on CTA pairs (half the barrier round trips
+  // per MMA: fprop / dgrad ~8% faster, wgrad's large groups ~9%; wgrad then
+  // keeps three stages by taking at most 256 groups a launch and transposing
+  // through 2 KB a warp), one on single CTAs.
   static constexpr int kSub = (CG == 2) ? ((MODE == kWgrad) ? kWgradSub : 2) : 1;
   static constexpr int kA1 = 128 * BK;  // A codes of a sub-stage: 16 KB
   // B codes per CTA and sub-stage: K-major kBRows x 128 B, MN-major 128-column chunks
@@ -78,10 +81,11 @@ struct CfgMX {
   static constexpr int kBAlloc = kSub * kB1;
   static_assert(kTN == 128 * kAtomsB, "a B tile is exactly the loaded scale atoms");
   static constexpr int kStageBytes = kABytes + kBAlloc + kSub * kSfBytes;
-  static constexpr int kStagingBytes = (MODE == kWgrad) ? kEpiWarps * 32 * 32 * 4 : 0;  // one 4 KB transpose per epilogue warp
+  static constexpr int kStagingBytes = (MODE == kWgrad) ? kEpiWarps * 32 * 16 * 4 : 0;  // one 2 KB transpose per epilogue warp
+  static constexpr int kMaxG = (MODE == kWgrad) ? kWgradMaxG : GL_MAX_GROUPS_MXFP8;  // groups per launch
   // as many stages as fit beside the barriers and the tile / scale prefixes
   // at the largest group count (at most six)
-  static constexpr int kFit = (232448 - 1024 - 256 - 2 * (GL_MAX_GROUPS_MXFP8 + 1) * 4 - kStagingBytes) / kStageBytes;
+  static constexpr int kFit = (232448 - 1024 - 256 - 2 * (kMaxG + 1) * 4 - kStagingBytes) / kStageBytes;
   static constexpr int kStages = kFit < 6 ? kFit : 6;
   static_assert(kStages >= 2, "pipeline too shallow");
   static constexpr int kTx = kABytes + kBAlloc + kSub * (kSfABytes + kAtomsB * 512);
@@ -91,7 +95,8 @@ struct CfgMX {
   static_assert((2 * kStages + 5) * 8 + 16 <= 256, "barrier area");
   static_assert(kSfCol0 + kSfSlots * kSfSlotCols <= 512, "TMEM columns");
   // dynamic shared memory at the largest group count (tile and scale prefixes), + alignment slack
-  static_assert(kPrefixOffset + 2 * (GL_MAX_GROUPS_MXFP8 + 1) * 4 + 1024 <= 232448, "shared memory");
+  static_assert(kPrefixOffset + 2 * (kMaxG + 1) * 4 + 1024 <= 232448, "shared memory");
+  static_assert(kPG <= kMaxG, "per-group launches");
   static_assert(kStageBytes % 1024 == 0, "alignment");
   // operand majorness in shared memory (1 = MN-major)
   static constexpr int kAMN = (MODE == kWgrad) ? 1 : 0;
@@ -675,12 +680,12 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
         // main_grad rows n0 + 0..31 (this warp's TMEM lanes) x columns k0 .. k0+127
         // (its half of the tile): copy them to registers and free the
         // accumulator, so the next tile's MMAs run while these sums leave.
-        // Each [32 x 32] fp32 chunk then goes through a 4 KB per-warp
+        // Each [32 x 16] fp32 piece then goes through a 2 KB per-warp
         // shared-memory transpose (16-byte pieces, XOR-swizzled: conflict-free
-        // both ways), so that 8 lanes cover one row's 128 contiguous bytes, and
+        // both ways), so that 4 lanes cover 64 contiguous bytes of a row, and
         // leaves as coalesced 16-byte vector reductions (accumulate) or stores
-        // (overwrite): full-line transactions, many in flight, no waits.
-        float* stg = reinterpret_cast<float*>(smem + C::kStagingOffset) + (warp - 2) * (32 * 32);
+        // (overwrite): full-sector transactions, many in flight, no waits.
+        float* stg = reinterpret_cast<float*>(smem + C::kStagingOffset) + (warp - 2) * (32 * 16);
         constexpr int kCols = TN / 2;  // columns of this warp (its half)
         constexpr int kChunks = kCols / 32;
         const int n0 = tl.mt * TMt + hr + q * 32;
@@ -702,27 +707,32 @@ __global__ void __launch_bounds__(CfgMX<MODE, CG>::kThreads, 1)
         release_acc();
         if (in_k) {
           float* gbase = PG ? pg.m(tl.g) : p.mg + static_cast<int64_t>(tl.g) * p.N * p.K;
-          const int sub = lane >> 3, piece = lane & 7;  // read side: row 4i + sub, 16-byte piece
-          float* mine = stg + lane * 32;
+          const int sub = lane >> 2, piece = lane & 3;  // read side: row 8i + sub, 16-byte piece
+          float* mine = stg + lane * 16;
+          const int wsw = (lane >> 1) & 3;  // write-side swizzle of this lane's row
 #pragma unroll
           for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(mine + ((j ^ (lane & 7)) << 2)) =
-                  make_uint4(r[c][4 * j], r[c][4 * j + 1], r[c][4 * j + 2], r[c][4 * j + 3]);
-            __syncwarp();
-            const int col = k0 + c * 32 + piece * 4;
+            for (int hh = 0; hh < 2; ++hh) {  // 16 of the chunk's 32 columns at a time
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int row = 4 * i + sub;
-              const uint4 v = *reinterpret_cast<const uint4*>(stg + row * 32 + ((piece ^ (row & 7)) << 2));
-              if (n0 + row < p.N) {
-                float* dst = gbase + static_cast<int64_t>(n0 + row) * p.K + col;
-                if (p.accumulate) red_add_v4(dst, v.x, v.y, v.z, v.w);
-                else *reinterpret_cast<uint4*>(dst) = v;
+              for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint4*>(mine + ((j ^ wsw) << 2)) =
+                    make_uint4(r[c][16 * hh + 4 * j], r[c][16 * hh + 4 * j + 1], r[c][16 * hh + 4 * j + 2],
+                               r[c][16 * hh + 4 * j + 3]);
+              __syncwarp();
+              const int col = k0 + c * 32 + hh * 16 + piece * 4;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int row = 8 * i + sub;
+                const uint4 v = *reinterpret_cast<const uint4*>(stg + row * 16 + ((piece ^ ((row >> 1) & 3)) << 2));
+                if (n0 + row < p.N) {
+                  float* dst = gbase + static_cast<int64_t>(n0 + row) * p.K + col;
+                  if (p.accumulate) red_add_v4(dst, v.x, v.y, v.z, v.w);
+                  else *reinterpret_cast<uint4*>(dst) = v;
+                }
               }
+              __syncwarp();  // the next piece overwrites the transpose buffer
             }
-            __syncwarp();  // the next chunk overwrites the transpose buffer
           }
         }
       }
@@ -880,12 +890,21 @@ gl_status mx_mode(const MxCall& c) {
       prm.mg = static_cast<float*>(const_cast<void*>(c.out_grouped.base));
     }
     if (!ok) return GL_ERR_UNSUPPORTED;
-    prm.offsets = c.offsets;
-    prm.G = c.G;
-    prm.g0 = 0;
     if (prm.has_bias) prm.bias = reinterpret_cast<const __nv_bfloat16*>(c.bias->base);
     MxPG<false> none{0};
-    return mx_launch<MODE, CG, false>(prm, none, c.G, c.stream);
+    // launches of at most kMaxG groups (wgrad: 256; the others take every group at once)
+    constexpr int kMaxG = CfgMX<MODE, CG>::kMaxG;
+    float* mg0 = prm.mg;
+    gl_status st = GL_OK;
+    for (int g0 = 0; g0 < c.G && st == GL_OK; g0 += kMaxG) {
+      const int cg = std::min(kMaxG, c.G - g0);
+      prm.offsets = c.offsets + g0;
+      prm.G = cg;
+      prm.g0 = g0;
+      if (MODE == kWgrad) prm.mg = mg0 + static_cast<int64_t>(g0) * c.N * c.K;
+      st = mx_launch<MODE, CG, false>(prm, none, cg, c.stream);
+    }
+    return st;
   }
   MxPG<true>* pga = new MxPG<true>;
   gl_status st = GL_OK;
