@@ -50,17 +50,17 @@ OP_SAMPLES = 50  # per-op medians are taken over at least this many steps
 # of the CUDA sources the capture ran.  When the sources have changed since,
 # the figures describe other kernels: the line then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "csrc_digest": "9ce8bc2146b2dc9f",
+    "csrc_digest": "f037632f4168708d",
     # the second step of `bench.py --steps 2 --warmup 3` under ncu (one pass,
     # gpu__time_duration / dram__bytes_read / dram__bytes_write per launch)
-    "bf16_g8": {"fwd": 1852200704, "dgrad": 2837817088, "wgrad": 5739353344,
-                "quant_x": 219744000, "quant_w": 1877931008, "quant_dy": 914936576,
-                "fwd_mx": 1006996480, "dgrad_mx": 1392577792, "wgrad_mx": 3656645120},
+    "bf16_g8": {"fwd": 1825746432, "dgrad": 2820858368, "wgrad": 5747676928,
+                "quant_x": 219182592, "quant_w": 1877729792, "quant_dy": 914067200,
+                "fwd_mx": 1006835200, "dgrad_mx": 1405178880, "wgrad_mx": 3657736704},
     # `bench.py --workload stacked_g128_ragged --steps 1 --warmup 1` under ncu
     # (the timed step's kernels; the MXFP8 wgrad from the warm-up step)
-    "stacked_g128_ragged": {"fwd": 5775737088, "dgrad": 4620293120, "wgrad": 15831860992,
-                            "quant_x": 1889802496, "quant_w": 7889447680, "quant_dy": 494449920,
-                            "fwd_mx": 2744198144, "dgrad_mx": 2817394432, "wgrad_mx": 14997782528},
+    "stacked_g128_ragged": {"fwd": 5596950272, "dgrad": 4619833600, "wgrad": 15660184320,
+                            "quant_x": 1890677760, "quant_w": 7898937856, "quant_dy": 493870336,
+                            "fwd_mx": 2672948224, "dgrad_mx": 2815816448, "wgrad_mx": 14946737664},
 }
 
 
