@@ -2,7 +2,7 @@
 
 The full-size GPU parity tests cannot run the whole fp64 products, so they
 compare sampled outputs against ``fwd_entry`` / ``dgrad_entry`` /
-``wgrad_entry`` and judge every group with ``rel_frobenius``.  These helpers
+``wgrad_entry`` and check every group with ``rel_frobenius``.  These helpers
 are pinned here against things other than themselves:
 
 * each entry helper against torch fp64 ``split`` -> ``F.linear`` -> ``cat``
